@@ -1,0 +1,7 @@
+"""CPU oracle for the MSA hot path: test infrastructure, not product code.
+
+Only the tests, the package smoke check and the benchmark's CPU-baseline /
+reference arm may import it.
+"""
+from .msa_oracle import (block_scores, select_blocks, boundary_gap, sparse_attention,  # noqa: F401
+                         merge_partials, msa_rows)
