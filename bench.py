@@ -1,0 +1,472 @@
+"""Benchmark of the MSA hot path on B200: tokens/s and roofline fractions.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole hot path over one batch of synthetic inputs:
+the default workload `msa_128k_1m` is a 131,072-token chunked prefill (8 chunks
+of 16,384 queries: indexer -> top-k -> block-major attention) followed by one
+decode step of 64 sequences at 131,072 tokens and one of 8 sequences at
+1,048,576 tokens (indexer -> top-k -> split-K attention), all in one layer,
+M3 head configuration (64 query / 4 KV heads, head_dim 128, indexer 8 x 64,
+k = 16).  `value` counts every query token of the step.
+
+With torchrun (N > 1) every rank runs its own replica (weak scaling: the
+units are independent sequences), timed between barriers; the slowest rank's
+time sets `value`.  `--impl reference` times the CPU oracle on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import configs, gen  # noqa: E402
+
+METRIC = "MSA tokens/s (prefill & decode) at 128K/1M ctx; % of HBM/tensor roofline"
+WORKLOADS = ("msa_128k_1m", "chunked_prefill_128k", "prefill_32k", "decode_128k", "decode_1m", "verify_ragged",
+             "tiny_prefill_2k")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ workload parts
+
+class Part:
+    """One batch through the three calls (indexer, top-k, attention)."""
+
+    def __init__(self, name, wl, caches, kind, out_rows=None):
+        import block_sparse_long_13_b200 as msa
+        self.msa = msa
+        self.name, self.wl, self.kind = name, wl, kind
+        dev = "cuda"
+        self.cfg = msa.Config(num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim,
+                              idx_heads=wl.idx_heads, idx_dim=wl.idx_dim, block_size=wl.block_size,
+                              topk=wl.topk)
+        self.batch = msa.Batch.make(wl.q_start, wl.ctx_len, wl.page_table, wl.num_pages, device=dev)
+        self.caches = caches
+        self.q = gen.query_rows(wl, gen.TID_Q, device=dev)
+        self.idx_q = gen.query_rows(wl, gen.TID_IDX_Q, device=dev)
+        T, G, nb = wl.total_q, wl.num_kv_heads, wl.max_blocks
+        self.scores = torch.empty((T, G, nb), dtype=torch.float32, device=dev)
+        self.sel = torch.empty((T, G, wl.topk), dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(self.q) if out_rows is None else out_rows
+        self.lse = torch.empty((T, wl.num_q_heads), dtype=torch.float32, device=dev)
+        wsb = (msa.prefill_workspace_bytes if kind == "prefill" else msa.decode_workspace_bytes)(self.cfg, self.batch)
+        self.ws_bytes = wsb
+        self.ws = None
+        self.launches = 7 if kind == "prefill" else 3
+        self.pos = wl.positions()
+
+    def run(self, ws, ev=None, stream=None):
+        m = self.msa
+        if ev is not None:
+            ev[0].record(stream)
+        m.index_scores(self.cfg, self.batch, self.idx_q, self.caches["idx_k"], self.scores)
+        if ev is not None:
+            ev[1].record(stream)
+        m.topk_blocks(self.cfg, self.batch, self.scores, self.sel)
+        if ev is not None:
+            ev[2].record(stream)
+        fn = m.attn_prefill if self.kind == "prefill" else m.attn_decode
+        fn(self.cfg, self.batch, self.q, self.caches["k"], self.caches["v"], self.sel, self.out, self.lse,
+           ws[:self.ws_bytes])
+        if ev is not None:
+            ev[3].record(stream)
+
+    # ---- algorithmic work (for the roofline), from the shapes and the selection
+    def index_work(self):
+        wl = self.wl
+        vis = (self.pos + 1).double()
+        if self.kind == "prefill":
+            return {"flops": float(vis.sum()) * 2 * wl.idx_dim * wl.idx_heads}
+        ctx = torch.tensor(wl.ctx_len, dtype=torch.float64)
+        return {"bytes": float(ctx.sum()) * wl.idx_heads * wl.idx_dim * 2}
+
+    def attn_work(self):
+        wl = self.wl
+        sel = self.sel.long().cpu()
+        pos = self.pos.view(-1, 1, 1)
+        vis = torch.clamp(pos - sel * wl.block_size + 1, 0, wl.block_size)
+        vis = torch.where(sel >= 0, vis, torch.zeros_like(vis))
+        keys = float(vis.sum())  # per (row, group)
+        G = wl.num_q_heads // wl.num_kv_heads
+        flops = keys * G * 4 * wl.head_dim
+        bytes_ = keys * 2 * wl.head_dim * 2 + self.q.numel() * 2 * 2
+        return {"flops": flops, "bytes": bytes_}
+
+    def topk_work(self):
+        cur = (self.pos // self.wl.block_size).double()
+        return {"bytes": float(cur.sum()) * self.wl.num_kv_heads * 4 + self.sel.numel() * 4}
+
+
+def build_parts(name):
+    """Device inputs of a workload: list of Part (in order) plus total queries."""
+    parts = []
+    if name in ("msa_128k_1m", "chunked_prefill_128k"):
+        chunks = configs.chunked_prefill_128k()
+        full = chunks[-1]
+        caches = {"k": gen.paged_cache(full, gen.TID_K, device="cuda"),
+                  "v": gen.paged_cache(full, gen.TID_V, device="cuda"),
+                  "idx_k": gen.paged_cache(full, gen.TID_IDX_K, device="cuda")}
+        out_all = torch.empty((8 * 16384, 64, 128), dtype=torch.bfloat16, device="cuda")
+        for c, wl in enumerate(chunks):
+            parts.append(Part(f"prefill128k/c{c}", wl, caches, "prefill", out_all[c * 16384:(c + 1) * 16384]))
+    if name in ("msa_128k_1m", "decode_128k", "decode_1m", "verify_ragged"):
+        for dn in (("decode_128k", "decode_1m") if name == "msa_128k_1m" else (name,)):
+            wl = configs.ALL[dn]()
+            caches = {"k": gen.paged_cache(wl, gen.TID_K, device="cuda"),
+                      "v": gen.paged_cache(wl, gen.TID_V, device="cuda"),
+                      "idx_k": gen.paged_cache(wl, gen.TID_IDX_K, device="cuda")}
+            parts.append(Part(dn, wl, caches, "decode"))
+    if name in ("prefill_32k", "tiny_prefill_2k"):
+        wl = configs.ALL[name]()
+        caches = {"k": gen.paged_cache(wl, gen.TID_K, device="cuda"),
+                  "v": gen.paged_cache(wl, gen.TID_V, device="cuda"),
+                  "idx_k": gen.paged_cache(wl, gen.TID_IDX_K, device="cuda")}
+        parts.append(Part(name, wl, caches, "prefill"))
+    return parts
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        load = [x for x in sm if mx and x > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ the oracle (CPU baseline / reference arm)
+
+def oracle_sample(seconds_target=15.0, max_rows=None):
+    """Time the CPU oracle on query rows drawn uniformly from the step's
+    131,072 prefill queries (the step's 72 decode rows are 0.05% of its
+    tokens).  Inputs come from the seeded generator (on the GPU when there is
+    one, untimed) and are copied to host memory; the timed part is the oracle
+    alone: indexer over every visible block, top-k, sparse attention."""
+    from oracle import msa_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    chunks = configs.chunked_prefill_128k()
+    full = chunks[-1]
+    L = full.ctx_len[0]
+    host = {}
+    for key, tid in (("idx_k", gen.TID_IDX_K), ("k", gen.TID_K), ("v", gen.TID_V)):
+        host[key] = gen.token_tensor(full, tid, 0, torch.arange(L), device=dev).float().cpu().numpy()
+    rng = np.random.default_rng(0)
+    picks = sorted(int(x) for x in rng.integers(0, L, size=512))
+    qrows = {}
+    done = 0
+    t_oracle = 0.0
+    for gpos in picks:
+        c = gpos // 16384
+        wl = chunks[c]
+        r = gpos - c * 16384
+        if c not in qrows:
+            qrows[c] = (gen.query_rows(wl, gen.TID_Q, device=dev).cpu(), gen.query_rows(wl, gen.TID_IDX_Q, device=dev).cpu())
+        q_all, iq_all = qrows[c]
+        pos = np.array([gpos])
+        t0 = time.perf_counter()
+        O.msa_rows(q_all[r:r + 1].float().numpy(), iq_all[r:r + 1].float().numpy(), host["k"], host["v"],
+                   host["idx_k"], pos, wl.num_kv_heads, wl.block_size, wl.topk, wl.max_blocks)
+        t_oracle += time.perf_counter() - t0
+        done += 1
+        if t_oracle > seconds_target or (max_rows and done >= max_rows):
+            break
+    return {"value": done / t_oracle, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{done} query rows drawn uniformly from the 131072-token prefill (indexer over every "
+                      f"visible block, top-k, sparse attention; float64 numpy), {t_oracle:.1f} s of oracle time"}
+
+
+# ------------------------------------------------------------------ main
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        rank = int(os.environ["RANK"])
+        local = int(os.environ.get("LOCAL_RANK", rank))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return rank, ws, local
+    return 0, 1, 0
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args, rank, ws):
+    if rank != 0:
+        return
+    steps = []
+    for _ in range(args.warmup):
+        oracle_sample(seconds_target=2.0, max_rows=4)
+    for _ in range(args.steps):
+        steps.append(oracle_sample(seconds_target=20.0 / max(1, args.steps)))
+    val = statistics.median(s["value"] for s in steps)
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
+            "config": {"workload": args.workload, "sample": steps[-1]["sample"]},
+            "cpu_baseline": dict(steps[-1], value=val),
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="msa_128k_1m", choices=WORKLOADS)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    rank, ws, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, rank, ws)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    import block_sparse_long_13_b200 as msa
+    msa.load_library()  # fails loudly when the CUDA library is missing
+
+    parts = build_parts(args.workload)
+    stream = torch.cuda.current_stream()
+    ws_bytes = max(p.ws_bytes for p in parts)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    tokens = sum(p.wl.total_q for p in parts)
+    nev = len(parts)
+
+    def step(evs=None):
+        for i, p in enumerate(parts):
+            p.run(workspace, None if evs is None else evs[i], stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = msa.device_status()
+    if st != msa.MSA_OK:
+        raise SystemExit(f"device status {st} after warm-up")
+
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nev)]
+           for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = max_over_ranks(ms, ws)
+    value = tokens * ws / (ms_max / 1e3)
+
+    # per-call device times (average over the timed steps) and algorithmic work
+    calls = {}
+    for i, p in enumerate(parts):
+        t_idx = statistics.mean(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps))
+        t_top = statistics.mean(evs[k][i][1].elapsed_time(evs[k][i][2]) for k in range(args.steps))
+        t_att = statistics.mean(evs[k][i][2].elapsed_time(evs[k][i][3]) for k in range(args.steps))
+        calls[p.name] = {"index_ms": t_idx, "topk_ms": t_top, "attn_ms": t_att,
+                         "index": p.index_work(), "attn": p.attn_work(), "topk": p.topk_work(), "kind": p.kind,
+                         "tokens": p.wl.total_q}
+    pk = peaks()
+    # dominant call type over the step
+    agg = {}
+    for name, c in calls.items():
+        for key in ("index", "topk", "attn"):
+            tag = f"{key}_{c['kind']}"
+            a = agg.setdefault(tag, {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0})
+            a["ms"] += c[f"{key}_ms"]
+            a["flops"] += c[key].get("flops", 0.0)
+            a["bytes"] += c[key].get("bytes", 0.0)
+            a["launches"] += 1
+    dom_tag, dom = max(agg.items(), key=lambda kv: kv[1]["ms"])
+    if dom_tag in ("index_prefill", "attn_prefill"):
+        ach = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        roof = {"kernel": dom_tag, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": None,
+                "peak_source": pk["source"] + " (burst bf16)", "launch_ms": dom["ms"] / dom["launches"]}
+    else:
+        ach = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+        roof = {"kernel": dom_tag, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"] + " (copy)",
+                "launch_ms": dom["ms"] / dom["launches"]}
+    fractions = {}
+    for tag, a in agg.items():
+        if a["ms"] <= 0:
+            continue
+        if "prefill" in tag and tag != "topk_prefill":
+            fractions[tag] = {"tflops": a["flops"] / a["ms"] / 1e9, "frac_of_measured_bf16":
+                              a["flops"] / a["ms"] / 1e9 / pk["bf16_tflops"], "ms_per_step": a["ms"]}
+        else:
+            gbs = a["bytes"] / a["ms"] / 1e6
+            fractions[tag] = {"gbs": gbs, "frac_of_measured_hbm": gbs / pk["hbm_gbs"],
+                              "frac_of_8tbs": gbs / 8000.0, "ms_per_step": a["ms"]}
+    parts_summary = {}
+    pre = [c for c in calls.values() if c["kind"] == "prefill"]
+    if pre:
+        t = sum(c["index_ms"] + c["topk_ms"] + c["attn_ms"] for c in pre)
+        parts_summary["prefill"] = {"tokens": sum(c["tokens"] for c in pre), "ms": t,
+                                    "tokens_per_s": sum(c["tokens"] for c in pre) / (t / 1e3)}
+    for name, c in calls.items():
+        if c["kind"] == "decode":
+            t = c["index_ms"] + c["topk_ms"] + c["attn_ms"]
+            parts_summary[name] = {"tokens": c["tokens"], "ms": t, "tokens_per_s": c["tokens"] / (t / 1e3)}
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host_in, host_out = [], []
+        for p in parts:
+            hin = {"q": p.q.cpu().pin_memory(), "idx_q": p.idx_q.cpu().pin_memory()}
+            host_in.append(hin)
+            host_out.append(torch.empty(p.out.shape, dtype=p.out.dtype).pin_memory())
+        new_kv = None
+        if parts[0].kind == "prefill":
+            # the prefill's own keys / values / indexer keys are inputs of the step too
+            cch = parts[0].caches
+            new_kv = {k: cch[k].cpu().pin_memory() for k in ("k", "v", "idx_k")}
+        h2d = sum(t.numel() * t.element_size() for h in host_in for t in h.values())
+        if new_kv is not None:
+            h2d += sum(t.numel() * t.element_size() for t in new_kv.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+        def e2e_step():
+            if new_kv is not None:
+                for key, t in new_kv.items():
+                    parts[0].caches[key].copy_(t, non_blocking=True)
+            for p, hin in zip(parts, host_in):
+                p.q.copy_(hin["q"], non_blocking=True)
+                p.idx_q.copy_(hin["idx_q"], non_blocking=True)
+            step()
+            for p, hout in zip(parts, host_out):
+                hout.copy_(p.out, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        ksteps = max(2, args.steps // 2)
+        for _ in range(ksteps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        ems = max_over_ranks(a0.elapsed_time(a1) / ksteps, ws)
+        e2e = {"value": tokens * ws / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": ems}
+    st = msa.device_status()
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
+                "config": {"workload": args.workload, "tokens_per_step": tokens,
+                           "parts": [p.name for p in parts], "l2": "inputs larger than L2 (no flush)",
+                           "heads": "64q/4kv, head_dim 128, indexer 8x64, block 128, k=16",
+                           "parallelism": f"replicas x{ws}"},
+                "roofline": roof, "fractions": fractions, "parts": parts_summary,
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+                "gpu_launches": sum(p.launches for p in parts) * args.steps,
+                "device_status": int(st)}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

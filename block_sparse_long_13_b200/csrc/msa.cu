@@ -1,0 +1,496 @@
+// C ABI of the MSA hot path: argument checks, TMA descriptors, launches.
+// Declarations and the contract of every entry point are in include/msa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/msa.h"
+#include "attn_decode.cuh"
+#include "attn_prefill.cuh"
+#include "common.cuh"
+#include "index_decode.cuh"
+#include "index_prefill.cuh"
+#include "topk.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+msa_status_t fail(msa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+#define CHECK_ARG(cond, ...) \
+  do {                       \
+    if (!(cond)) return fail(MSA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+#define CHECK_SUP(cond, ...) \
+  do {                       \
+    if (!(cond)) return fail(MSA_ERR_UNSUPPORTED, __VA_ARGS__); \
+  } while (0)
+#define CUDA_TRY(call)                                                                         \
+  do {                                                                                         \
+    cudaError_t e_ = (call);                                                                   \
+    if (e_ != cudaSuccess) return fail(MSA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+float softmax_scale(const msa_config_t* c) {
+  return c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / std::sqrt(static_cast<float>(c->head_dim));
+}
+
+msa_status_t check_config(const msa_config_t* c) {
+  CHECK_ARG(c != nullptr, "cfg is NULL");
+  CHECK_ARG(c->num_q_heads > 0 && c->num_kv_heads > 0 && c->idx_heads > 0 && c->topk > 0,
+            "head counts and topk must be positive");
+  CHECK_ARG(c->num_q_heads % c->num_kv_heads == 0, "num_q_heads must be a multiple of num_kv_heads");
+  CHECK_ARG(c->idx_heads % c->num_kv_heads == 0, "idx_heads must be a multiple of num_kv_heads");
+  CHECK_SUP(c->num_q_heads / c->num_kv_heads == 16, "this build needs 16 query heads per KV head");
+  CHECK_SUP(c->idx_heads / c->num_kv_heads <= 4, "at most 4 indexer heads per KV group");
+  CHECK_SUP(c->idx_heads <= 16, "at most 16 indexer heads");
+  CHECK_SUP(c->head_dim == 128, "head_dim must be 128");
+  CHECK_SUP(c->idx_dim == 64, "idx_dim must be 64");
+  CHECK_SUP(c->block_size == 128, "block_size must be 128");
+  CHECK_SUP(c->topk <= 64, "topk must be <= 64");
+  CHECK_ARG(!(c->softmax_scale != c->softmax_scale), "softmax_scale is NaN");
+  return MSA_OK;
+}
+
+msa_status_t check_batch(const msa_batch_t* b) {
+  CHECK_ARG(b != nullptr, "batch is NULL");
+  CHECK_ARG(b->num_seqs > 0, "num_seqs must be positive");
+  CHECK_ARG(b->total_q >= 0, "total_q must be >= 0");
+  CHECK_ARG(b->max_blocks_per_seq > 0, "max_blocks_per_seq must be positive");
+  CHECK_SUP(b->max_blocks_per_seq <= 16384, "max_blocks_per_seq must be <= 16384");
+  CHECK_ARG(b->max_q_per_seq > 0, "max_q_per_seq must be positive");
+  CHECK_ARG(b->num_pages > 0, "num_pages must be positive");
+  CHECK_ARG(b->q_start && b->ctx_len && b->page_table, "batch index arrays must not be NULL");
+  CHECK_SUP(b->total_q < (1 << 25), "total_q must be < 2^25");
+  return MSA_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle
+msa_status_t make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                      const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return MSA_OK;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+msa_status_t launched() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MSA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return MSA_OK;
+}
+
+// ---------------------------------------------------------------- workspace plans
+struct PrefillWs {
+  size_t counts, offsets, tile_offsets, cursor, total_tiles, entries, part_lse, part_o, bytes;
+  long nbuckets;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+PrefillWs prefill_plan(const msa_config_t* c, const msa_batch_t* b) {
+  PrefillWs w{};
+  w.nbuckets = static_cast<long>(b->num_seqs) * c->num_kv_heads * b->max_blocks_per_seq;
+  size_t o = 0;
+  auto take = [&](size_t n) { size_t at = o; o = align_up(o + n, 256); return at; };
+  w.counts = take(w.nbuckets * 4);
+  w.offsets = take((w.nbuckets + 1) * 4);
+  w.tile_offsets = take((w.nbuckets + 1) * 4);
+  w.cursor = take(w.nbuckets * 4);
+  w.total_tiles = take(16);
+  const size_t ent = static_cast<size_t>(b->total_q) * c->num_kv_heads * c->topk;
+  w.entries = take(ent * 4);
+  w.part_lse = take(static_cast<size_t>(b->total_q) * c->num_q_heads * c->topk * 4);
+  w.part_o = take(static_cast<size_t>(b->total_q) * c->topk * c->num_q_heads * c->head_dim * 2);
+  w.bytes = o;
+  return w;
+}
+
+int decode_splits(const msa_config_t* c, const msa_batch_t* b) {
+  const long units = static_cast<long>(b->total_q) * c->num_kv_heads;
+  if (units <= 0) return 1;
+  long want = (4L * 148 + units - 1) / units;  // aim at ~4 CTAs per SM of a 148-SM B200
+  if (want < 1) want = 1;
+  if (want > c->topk) want = c->topk;
+  return static_cast<int>(want);
+}
+
+struct DecodeWs {
+  size_t counters, part_lse, part_o, bytes;
+  int nsplit;
+};
+
+DecodeWs decode_plan(const msa_config_t* c, const msa_batch_t* b) {
+  DecodeWs w{};
+  w.nsplit = decode_splits(c, b);
+  const size_t units = static_cast<size_t>(b->total_q) * c->num_kv_heads;
+  size_t o = 0;
+  auto take = [&](size_t n) { size_t at = o; o = align_up(o + n, 256); return at; };
+  w.counters = take(units * 4);
+  w.part_lse = take(units * w.nsplit * 16 * 4);
+  w.part_o = take(units * w.nsplit * 16 * 128 * 4);
+  w.bytes = o;
+  return w;
+}
+
+__global__ void wait_forever_probe_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    msa::mbar_init(&bar, 1);
+    msa::fence_mbar_init();
+    msa::mbar_wait(&bar, 0, &abort_flag);  // nothing arrives: must time out
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* msa_status_string(msa_status_t s) {
+  switch (s) {
+    case MSA_OK: return "ok";
+    case MSA_ERR_INVALID_ARG: return "invalid argument";
+    case MSA_ERR_UNSUPPORTED: return "unsupported size or layout";
+    case MSA_ERR_CUDA: return "CUDA error";
+    case MSA_ERR_TIMEOUT: return "device wait timed out";
+    case MSA_ERR_DEVICE_BOUNDS: return "device found an out-of-range index";
+  }
+  return "unknown status";
+}
+
+const char* msa_last_error(void) { return g_msg; }
+
+int32_t msa_version(void) { return 100; }
+
+size_t msa_prefill_workspace_bytes(const msa_config_t* cfg, const msa_batch_t* batch) {
+  if (check_config(cfg) != MSA_OK || check_batch(batch) != MSA_OK) return 0;
+  return prefill_plan(cfg, batch).bytes;
+}
+
+size_t msa_decode_workspace_bytes(const msa_config_t* cfg, const msa_batch_t* batch) {
+  if (check_config(cfg) != MSA_OK || check_batch(batch) != MSA_OK) return 0;
+  return decode_plan(cfg, batch).bytes;
+}
+
+msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
+                              const void* idx_k_cache, float* block_scores, cudaStream_t stream) {
+  msa_status_t st;
+  if ((st = check_config(cfg)) != MSA_OK) return st;
+  if ((st = check_batch(batch)) != MSA_OK) return st;
+  CHECK_ARG(idx_q && idx_k_cache && block_scores, "idx_q, idx_k_cache and block_scores must not be NULL");
+  CHECK_ARG(aligned16(idx_q) && aligned16(idx_k_cache) && aligned16(block_scores), "pointers must be 16-byte aligned");
+  if (batch->total_q == 0) return MSA_OK;
+  const int Hi = cfg->idx_heads, Hkv = cfg->num_kv_heads, hg = Hi / Hkv;
+  CUtensorMap tk;
+  {
+    const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
+    const uint64_t strides[3] = {128, 128 * 128, static_cast<uint64_t>(Hi) * 128 * 128};
+    const uint32_t box[4] = {64, 128, static_cast<uint32_t>(hg), 1};
+    if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box)) != MSA_OK) return st;
+  }
+  const int sms = num_sms();
+  if (batch->max_q_per_seq <= msa::IDXD_MAXQ) {
+    CHECK_SUP(batch->num_seqs <= msa::IDXD_MAXSEQ, "at most %d sequences per streaming indexer call",
+              msa::IDXD_MAXSEQ);
+    msa::IdxDecodeArgs a{};
+    a.idx_q = static_cast<const __nv_bfloat16*>(idx_q);
+    a.scores = block_scores;
+    a.q_start = batch->q_start;
+    a.ctx_len = batch->ctx_len;
+    a.page_table = batch->page_table;
+    a.num_seqs = batch->num_seqs;
+    a.max_blocks = batch->max_blocks_per_seq;
+    a.num_pages = batch->num_pages;
+    a.Hi = Hi;
+    a.Hkv = Hkv;
+    a.hg = hg;
+    a.block_size = cfg->block_size;
+    a.stage_bytes = hg * 128 * 64 * 2;
+    a.stages = std::min(16, msa::IDXD_RING_BYTES / a.stage_bytes);
+    const int smem = a.stages * a.stage_bytes + 1024;
+    CUDA_TRY(set_smem(msa::index_decode_kernel, smem));
+    msa::index_decode_kernel<<<sms, msa::IDXD_THREADS, smem, stream>>>(tk, a);
+    return launched();
+  }
+  CHECK_SUP(batch->num_seqs <= msa::IDXP_MAXSEQ, "at most %d sequences per tensor-core indexer call",
+            msa::IDXP_MAXSEQ);
+  CUtensorMap tq;
+  {
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->total_q)};
+    const uint64_t strides[2] = {128, static_cast<uint64_t>(Hi) * 128};
+    const uint32_t box[3] = {64, 1, 128};
+    if ((st = make_map(&tq, idx_q, 3, dims, strides, box)) != MSA_OK) return st;
+  }
+  msa::IdxPrefillArgs a{};
+  a.scores = block_scores;
+  a.q_start = batch->q_start;
+  a.ctx_len = batch->ctx_len;
+  a.page_table = batch->page_table;
+  a.num_seqs = batch->num_seqs;
+  a.total_q = batch->total_q;
+  a.max_blocks = batch->max_blocks_per_seq;
+  a.num_pages = batch->num_pages;
+  a.Hi = Hi;
+  a.Hkv = Hkv;
+  a.hg = hg;
+  a.block_size = cfg->block_size;
+  const int tile_bytes = hg * 128 * 64 * 2;
+  a.stages = std::min(8, (200 * 1024 - tile_bytes) / tile_bytes);
+  a.nbuf = std::max(1, 4 / hg);
+  CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
+  const int smem = tile_bytes * (1 + a.stages) + 1024;
+  CUDA_TRY(set_smem(msa::index_prefill_kernel, smem));
+  msa::index_prefill_kernel<<<sms, msa::IDXP_THREADS, smem, stream>>>(tq, tk, a);
+  return launched();
+}
+
+msa_status_t msa_topk_blocks(const msa_config_t* cfg, const msa_batch_t* batch, const float* block_scores,
+                             int32_t* block_idx, cudaStream_t stream) {
+  msa_status_t st;
+  if ((st = check_config(cfg)) != MSA_OK) return st;
+  if ((st = check_batch(batch)) != MSA_OK) return st;
+  CHECK_ARG(block_scores && block_idx, "block_scores and block_idx must not be NULL");
+  if (batch->total_q == 0) return MSA_OK;
+  const long rows = static_cast<long>(batch->total_q) * cfg->num_kv_heads;
+  const int nb = batch->max_blocks_per_seq;
+  const int Hkv = cfg->num_kv_heads, k = cfg->topk, bs = cfg->block_size;
+#define TOPK_ARGS block_scores, block_idx, batch->q_start, batch->ctx_len, batch->num_seqs, batch->total_q, Hkv, nb, k, bs
+  if (nb <= 256) {
+    msa::topk_blocks_kernel<1, 8><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(TOPK_ARGS);
+  } else if (nb <= 1024) {
+    msa::topk_blocks_kernel<1, 32><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(TOPK_ARGS);
+  } else if (nb <= 2048) {
+    msa::topk_blocks_kernel<2, 32><<<static_cast<unsigned>(rows), 64, 0, stream>>>(TOPK_ARGS);
+  } else if (nb <= 4096) {
+    msa::topk_blocks_kernel<4, 32><<<static_cast<unsigned>(rows), 128, 0, stream>>>(TOPK_ARGS);
+  } else if (nb <= 8192) {
+    msa::topk_blocks_kernel<8, 32><<<static_cast<unsigned>(rows), 256, 0, stream>>>(TOPK_ARGS);
+  } else {
+    msa::topk_blocks_kernel<16, 32><<<static_cast<unsigned>(rows), 512, 0, stream>>>(TOPK_ARGS);
+  }
+#undef TOPK_ARGS
+  return launched();
+}
+
+msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch, const void* q, const void* k_cache,
+                              const void* v_cache, const int32_t* block_idx, void* out, float* lse, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+  msa_status_t st;
+  if ((st = check_config(cfg)) != MSA_OK) return st;
+  if ((st = check_batch(batch)) != MSA_OK) return st;
+  CHECK_ARG(q && k_cache && v_cache && block_idx && out, "q, caches, block_idx and out must not be NULL");
+  CHECK_ARG(aligned16(q) && aligned16(k_cache) && aligned16(v_cache) && aligned16(out) && aligned16(workspace),
+            "pointers must be 16-byte aligned");
+  const PrefillWs w = prefill_plan(cfg, batch);
+  CHECK_ARG(workspace != nullptr && workspace_bytes >= w.bytes, "workspace too small: %zu bytes needed", w.bytes);
+  CHECK_SUP(w.nbuckets < (1L << 31), "too many (sequence, group, block) buckets");
+  if (batch->total_q == 0) return MSA_OK;
+  char* ws = static_cast<char*>(workspace);
+  const int Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, k = cfg->topk;
+
+  msa::SchedArgs s{};
+  s.block_idx = block_idx;
+  s.q_start = batch->q_start;
+  s.ctx_len = batch->ctx_len;
+  s.counts = reinterpret_cast<int*>(ws + w.counts);
+  s.offsets = reinterpret_cast<int*>(ws + w.offsets);
+  s.tile_offsets = reinterpret_cast<int*>(ws + w.tile_offsets);
+  s.cursor = reinterpret_cast<int*>(ws + w.cursor);
+  s.entries = reinterpret_cast<int*>(ws + w.entries);
+  s.total_tiles = reinterpret_cast<int*>(ws + w.total_tiles);
+  s.num_seqs = batch->num_seqs;
+  s.total_q = batch->total_q;
+  s.Hkv = Hkv;
+  s.topk = k;
+  s.max_blocks = batch->max_blocks_per_seq;
+  s.block_size = cfg->block_size;
+  s.nbuckets = static_cast<int>(w.nbuckets);
+  CUDA_TRY(cudaMemsetAsync(s.counts, 0, w.nbuckets * 4, stream));
+  const unsigned sgrid = static_cast<unsigned>((batch->total_q + msa::SCHED_ROWS - 1) / msa::SCHED_ROWS);
+  const int ssmem = w.nbuckets <= msa::SCHED_SMEM_BUCKETS ? static_cast<int>(3 * w.nbuckets * 4) : 0;
+  msa::sched_count_scatter_kernel<<<sgrid, 256, ssmem, stream>>>(s, 0);
+  if ((st = launched()) != MSA_OK) return st;
+  msa::sched_scan_kernel<<<1, 1024, 0, stream>>>(s);
+  if ((st = launched()) != MSA_OK) return st;
+  msa::sched_count_scatter_kernel<<<sgrid, 256, ssmem, stream>>>(s, 1);
+  if ((st = launched()) != MSA_OK) return st;
+
+  CUtensorMap tq, tk, tv, tpo;
+  {
+    const uint64_t dims[2] = {128, static_cast<uint64_t>(batch->total_q) * Hq};
+    const uint64_t strides[1] = {256};
+    const uint32_t box[2] = {64, 16};
+    if ((st = make_map(&tq, q, 2, dims, strides, box)) != MSA_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {128, static_cast<uint64_t>(batch->num_pages) * Hkv * 128};
+    const uint64_t strides[1] = {256};
+    const uint32_t box[2] = {64, 128};
+    if ((st = make_map(&tk, k_cache, 2, dims, strides, box)) != MSA_OK) return st;
+    if ((st = make_map(&tv, v_cache, 2, dims, strides, box)) != MSA_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {128, static_cast<uint64_t>(batch->total_q) * k * Hq};
+    const uint64_t strides[1] = {256};
+    const uint32_t box[2] = {64, 16};
+    if ((st = make_map(&tpo, ws + w.part_o, 2, dims, strides, box)) != MSA_OK) return st;
+  }
+  msa::AttnPrefillArgs a{};
+  a.q_start = batch->q_start;
+  a.ctx_len = batch->ctx_len;
+  a.page_table = batch->page_table;
+  a.offsets = s.offsets;
+  a.tile_offsets = s.tile_offsets;
+  a.entries = s.entries;
+  a.total_tiles = s.total_tiles;
+  a.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
+  a.num_seqs = batch->num_seqs;
+  a.total_q = batch->total_q;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.topk = k;
+  a.max_blocks = batch->max_blocks_per_seq;
+  a.num_pages = batch->num_pages;
+  a.block_size = cfg->block_size;
+  a.nbuckets = s.nbuckets;
+  a.scale_log2 = softmax_scale(cfg) * 1.4426950408889634f;
+  CUDA_TRY(set_smem(msa::attn_prefill_kernel, msa::ATTP_SMEM));
+  msa::attn_prefill_kernel<<<num_sms(), msa::ATTP_THREADS, msa::ATTP_SMEM, stream>>>(tq, tk, tv, tpo, a);
+  if ((st = launched()) != MSA_OK) return st;
+
+  msa::MergeArgs m{};
+  m.part_o = reinterpret_cast<const __nv_bfloat16*>(ws + w.part_o);
+  m.part_lse = a.part_lse;
+  m.block_idx = block_idx;
+  m.out = static_cast<__nv_bfloat16*>(out);
+  m.lse = lse;
+  m.total_q = batch->total_q;
+  m.Hq = Hq;
+  m.Hkv = Hkv;
+  m.topk = k;
+  msa::attn_merge_kernel<<<static_cast<unsigned>(batch->total_q) * Hkv, 256, 0, stream>>>(m);
+  return launched();
+}
+
+msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, const void* q, const void* k_cache,
+                             const void* v_cache, const int32_t* block_idx, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+  msa_status_t st;
+  if ((st = check_config(cfg)) != MSA_OK) return st;
+  if ((st = check_batch(batch)) != MSA_OK) return st;
+  CHECK_ARG(q && k_cache && v_cache && block_idx && out, "q, caches, block_idx and out must not be NULL");
+  CHECK_ARG(aligned16(q) && aligned16(k_cache) && aligned16(v_cache) && aligned16(out) && aligned16(workspace),
+            "pointers must be 16-byte aligned");
+  const DecodeWs w = decode_plan(cfg, batch);
+  CHECK_ARG(workspace != nullptr && workspace_bytes >= w.bytes, "workspace too small: %zu bytes needed", w.bytes);
+  if (batch->total_q == 0) return MSA_OK;
+  char* ws = static_cast<char*>(workspace);
+  msa::AttnDecodeArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  a.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  a.block_idx = block_idx;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.q_start = batch->q_start;
+  a.ctx_len = batch->ctx_len;
+  a.page_table = batch->page_table;
+  a.part_o = reinterpret_cast<float*>(ws + w.part_o);
+  a.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
+  a.counters = reinterpret_cast<int*>(ws + w.counters);
+  a.num_seqs = batch->num_seqs;
+  a.total_q = batch->total_q;
+  a.Hq = cfg->num_q_heads;
+  a.Hkv = cfg->num_kv_heads;
+  a.topk = cfg->topk;
+  a.max_blocks = batch->max_blocks_per_seq;
+  a.num_pages = batch->num_pages;
+  a.block_size = cfg->block_size;
+  a.nsplit = w.nsplit;
+  a.scale_log2 = softmax_scale(cfg) * 1.4426950408889634f;
+  const size_t units = static_cast<size_t>(batch->total_q) * cfg->num_kv_heads;
+  CUDA_TRY(cudaMemsetAsync(a.counters, 0, units * 4, stream));
+  msa::attn_decode_kernel<<<static_cast<unsigned>(units * w.nsplit), msa::ATTD_THREADS, 0, stream>>>(a);
+  return launched();
+}
+
+msa_status_t msa_get_device_status(cudaStream_t stream) {
+  CUDA_TRY(cudaStreamSynchronize(stream));
+  unsigned int word = 0, zero = 0;
+  CUDA_TRY(cudaMemcpyFromSymbol(&word, msa::g_error, sizeof(word)));
+  CUDA_TRY(cudaMemcpyToSymbol(msa::g_error, &zero, sizeof(zero)));
+  if (word & msa::MSA_DEV_TIMEOUT) return fail(MSA_ERR_TIMEOUT, "a device-side wait timed out");
+  if (word & msa::MSA_DEV_BOUNDS) return fail(MSA_ERR_DEVICE_BOUNDS, "the device found an out-of-range index");
+  return MSA_OK;
+}
+
+msa_status_t msa_set_wait_limit_ns(uint64_t ns) {
+  CHECK_ARG(ns > 0, "the wait limit must be positive");
+  unsigned long long v = ns;
+  CUDA_TRY(cudaMemcpyToSymbol(msa::g_wait_limit_ns, &v, sizeof(v)));
+  return MSA_OK;
+}
+
+msa_status_t msa_debug_wait_timeout(cudaStream_t stream) {
+  wait_forever_probe_kernel<<<1, 32, 0, stream>>>();
+  return launched();
+}
+
+}  // extern "C"

@@ -1,0 +1,186 @@
+/*
+ * msa.h - C ABI of the MiniMax Sparse Attention (MSA) hot path for B200 (sm_100a).
+ *
+ * The method (sources: "MiniMax M3: 1M-token multimodal reasoning model now
+ * available with NVIDIA and vLLM support", daily.dev, sections "Summary" and
+ * "What makes M3 different"; "MiniMax-M3", inteligile model page, table
+ * "Checked in its code"; "MiniMax M3 in vLLM: Day-0-Unterstuetzung ...",
+ * 24-ai.news; "Serving AI agents at scale ...", shaam.blog, section "What
+ * makes MiniMax M3 different from other open-weight models?"):
+ * the KV sequence is cut into 128-token blocks; a lightweight indexer scores
+ * every causally visible block for each query and GQA group; the top-k blocks
+ * are kept; GQA attention (64 query heads over 4 KV heads) runs only over the
+ * kept, uncompressed blocks.
+ *
+ * Readings this library fixes where the pages are silent: block score = sum
+ * over the group's indexer heads of the max over the block's visible keys of
+ * the raw dot product; the query's own block is always kept; ties go to the
+ * lower block id; softmax scale 1/sqrt(head_dim) unless given.
+ *
+ * CONVENTIONS (all entry points)
+ *   - Every pointer argument except `cfg`/`batch` themselves and the host
+ *     fields of msa_batch_t is a DEVICE pointer on the current CUDA device.
+ *   - The caller owns all memory.  No entry point allocates device memory;
+ *     scratch space is passed in as `workspace`.
+ *   - Work is enqueued on `stream`; nothing synchronises the host except
+ *     msa_get_device_status().
+ *   - Arguments are checked before anything is launched; a failed check
+ *     returns MSA_ERR_INVALID_ARG / MSA_ERR_UNSUPPORTED and launches nothing
+ *     (msa_last_error() tells why).  A failed launch returns MSA_ERR_CUDA.
+ *   - Index errors found on the device (page id outside [0, num_pages), a
+ *     selected block after the query's block, more queries per sequence than
+ *     declared) and bounded waits that ran out are recorded in a device error
+ *     word and reported by msa_get_device_status(); the kernels skip the bad
+ *     access instead of faulting.
+ *
+ * LAYOUTS (row-major, bf16 = IEEE bfloat16, fp32 = IEEE float)
+ *   idx_q        bf16 [total_q][idx_heads][idx_dim]
+ *   idx_k_cache  bf16 [num_pages][idx_heads][block_size][idx_dim]
+ *   q            bf16 [total_q][num_q_heads][head_dim]
+ *   k_cache      bf16 [num_pages][num_kv_heads][block_size][head_dim]   (v_cache alike)
+ *   block_scores fp32 [total_q][num_kv_heads][max_blocks_per_seq]
+ *   block_idx    int32 [total_q][num_kv_heads][topk]   ascending ids, -1 padded
+ *   out          bf16 [total_q][num_q_heads][head_dim]
+ *   lse          fp32 [total_q][num_q_heads]  (natural log; may be NULL)
+ *   Query row t belongs to sequence s with q_start[s] <= t < q_start[s+1];
+ *   its position is p = ctx_len[s] - (q_start[s+1] - q_start[s]) + (t - q_start[s]),
+ *   i.e. the call's queries are the last tokens of the context, whose keys
+ *   are already in the caches.  Key block b of sequence s lives in physical
+ *   page page_table[s][b].  A prefill is the same call with an identity
+ *   page table.
+ *
+ * Supported sizes: head_dim 128, idx_dim 64, block_size 128,
+ * num_q_heads = 16 * num_kv_heads, idx_heads a multiple of num_kv_heads with
+ * at most 4 indexer heads per group, 1 <= topk <= 64, max_blocks_per_seq <=
+ * 16384 (2M tokens).  Pointers must be 16-byte aligned.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,  /* a pointer, size or layout argument is wrong        */
+  MSA_ERR_UNSUPPORTED = 2,  /* valid, but outside the sizes this build handles    */
+  MSA_ERR_CUDA = 3,         /* a CUDA runtime / driver call failed                 */
+  MSA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (status query)   */
+  MSA_ERR_DEVICE_BOUNDS = 5 /* the device found an out-of-range index (status)     */
+} msa_status_t;
+
+typedef struct {
+  int32_t num_q_heads;   /* H_q  (64 in the pages' configuration)                  */
+  int32_t num_kv_heads;  /* H_kv (4); H_q / H_kv query heads share one KV head      */
+  int32_t head_dim;      /* 128                                                     */
+  int32_t idx_heads;     /* indexer heads H_i, split contiguously over the KV groups */
+  int32_t idx_dim;       /* indexer head dim, 64                                    */
+  int32_t block_size;    /* tokens per KV block = tokens per cache page, 128        */
+  int32_t topk;          /* blocks kept per (query, group), current block included   */
+  float softmax_scale;   /* <= 0 selects 1 / sqrt(head_dim)                          */
+} msa_config_t;
+
+typedef struct {
+  int32_t num_seqs;           /* host: sequences in the batch                       */
+  int32_t total_q;            /* host: query rows in the call = q_start[num_seqs]   */
+  int32_t max_blocks_per_seq; /* host: row width of page_table and block_scores      */
+  int32_t max_q_per_seq;      /* host: upper bound of any sequence's query count     */
+  int32_t num_pages;          /* host: pages in every cache (page ids are < this)    */
+  const int32_t* q_start;     /* device [num_seqs + 1], q_start[0] = 0, non-decreasing */
+  const int32_t* ctx_len;     /* device [num_seqs], context length incl. this call's queries */
+  const int32_t* page_table;  /* device [num_seqs][max_blocks_per_seq]               */
+} msa_batch_t;
+
+/*
+ * Indexer block scores.  For query row t (position p), KV group g and block
+ * b <= p / block_size:
+ *   block_scores[t][g][b] = sum_{h in heads(g)} max_{j in b, j <= p} idx_q[t][h] . idx_k[j][h]
+ * with heads(g) = {g*H_i/H_kv, ..., (g+1)*H_i/H_kv - 1}, accumulated in fp32
+ * from bf16 products.  Entries b > p / block_size are left undefined (the
+ * call may write -inf there or leave them untouched).
+ * (inteligile "MiniMax-M3", row "Indexer-selected sparse attention":
+ * per-head key scores pooled into blocks; 24-ai.news: every query or GQA
+ * query group scores all available blocks with lightweight indexer kernels.)
+ * Calls with max_q_per_seq <= 8 stream the pages (decode / verify); larger
+ * ones run the tensor-core form.
+ */
+msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
+                              const void* idx_k_cache, float* block_scores, cudaStream_t stream);
+
+/*
+ * Top-k block selection per (query row, group).  cur = p / block_size is
+ * always kept; the other topk-1 slots take the best blocks b < cur with a
+ * finite score, ranked by (score descending, b ascending); a -inf score is
+ * never kept.  Written ascending and padded with -1 to topk entries.
+ * (inteligile "MiniMax-M3", row "Indexer-selected sparse attention":
+ * k = min(topk_blocks, #blocks), -inf-scored slots reported as -1.)
+ * Reads block_scores[t][g][0 .. cur-1] only.  Deterministic.
+ */
+msa_status_t msa_topk_blocks(const msa_config_t* cfg, const msa_batch_t* batch, const float* block_scores,
+                             int32_t* block_idx, cudaStream_t stream);
+
+/*
+ * Sparse GQA attention, block-major ("KV outer, gather Q": shaam.blog,
+ * section "What makes MiniMax M3 different ..."; daily.dev, "Serving
+ * options": KV-block-major prefill scheduling).  Query head h of row t uses
+ * KV head g = h / (H_q / H_kv) and the keys j <= p of the blocks in
+ * block_idx[t][g][:]:
+ *   out[t][h] = sum_j softmax_j(scale * q[t][h] . k[j][g]) v[j][g],
+ *   lse[t][h] = log sum_j exp(scale * q[t][h] . k[j][g])
+ * (plain softmax, no sink, no output gate: inteligile rows "Grouped-query
+ * attention", "Learnable attention sink", "Gated attention output").
+ * Each selected block is loaded once per CTA run; per-(row, head, slot)
+ * partial results go to `workspace` and are merged by log-sum-exp.
+ * `workspace` must hold msa_prefill_workspace_bytes(cfg, batch) bytes.
+ */
+msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch, const void* q,
+                              const void* k_cache, const void* v_cache, const int32_t* block_idx, void* out,
+                              float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Same result as msa_attn_prefill, organised for few queries per sequence:
+ * one CTA per (row, group, split of the selected slots), online softmax
+ * inside a split and a log-sum-exp merge of the splits.  `workspace` must
+ * hold msa_decode_workspace_bytes(cfg, batch) bytes; its first
+ * total_q * num_kv_heads int32 counters are cleared by the call itself.
+ */
+msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, const void* q,
+                             const void* k_cache, const void* v_cache, const int32_t* block_idx, void* out,
+                             float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace sizes (bytes) for the two attention calls; only the host fields of
+ * `batch` are read.  0 means the arguments are invalid. */
+size_t msa_prefill_workspace_bytes(const msa_config_t* cfg, const msa_batch_t* batch);
+size_t msa_decode_workspace_bytes(const msa_config_t* cfg, const msa_batch_t* batch);
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word: MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_DEVICE_BOUNDS (MSA_ERR_CUDA if the
+ * stream itself reports an error). */
+msa_status_t msa_get_device_status(cudaStream_t stream);
+
+/* Sets the wall-clock limit of every device-side wait on the current device
+ * (default 2 s); used by tests of the timeout path.  0 is rejected. */
+msa_status_t msa_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook for the timeout path: launches one CTA that waits on an mbarrier
+ * nothing will ever complete; it must give up after the wait limit, record
+ * MSA_ERR_TIMEOUT and exit.  Never faults. */
+msa_status_t msa_debug_wait_timeout(cudaStream_t stream);
+
+const char* msa_status_string(msa_status_t status);
+/* Message of the last failed call on this host thread ("" if none). */
+const char* msa_last_error(void);
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int32_t msa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */
