@@ -37,7 +37,7 @@ from workloads import configs, gen  # noqa: E402
 
 METRIC = "MSA tokens/s (prefill & decode) at 128K/1M ctx; % of HBM/tensor roofline"
 WORKLOADS = ("msa_128k_1m", "chunked_prefill_128k", "prefill_32k", "decode_128k", "decode_1m", "verify_ragged",
-             "tiny_prefill_2k")
+             "tiny_prefill_2k", "prefill_8k", "prefill_128k_last_chunk")
 
 
 def peaks():
@@ -79,19 +79,21 @@ class Part:
         self.launches = 7 if kind == "prefill" else 3
         self.pos = wl.positions()
 
-    def run(self, ws, ev=None, stream=None):
+    def run(self, ws, ev=None, stream=None, stop_after="attn"):
         m = self.msa
         if ev is not None:
             ev[0].record(stream)
         m.index_scores(self.cfg, self.batch, self.idx_q, self.caches["idx_k"], self.scores)
         if ev is not None:
             ev[1].record(stream)
-        m.topk_blocks(self.cfg, self.batch, self.scores, self.sel)
+        if stop_after != "index":
+            m.topk_blocks(self.cfg, self.batch, self.scores, self.sel)
         if ev is not None:
             ev[2].record(stream)
-        fn = m.attn_prefill if self.kind == "prefill" else m.attn_decode
-        fn(self.cfg, self.batch, self.q, self.caches["k"], self.caches["v"], self.sel, self.out, self.lse,
-           ws[:self.ws_bytes])
+        if stop_after == "attn":
+            fn = m.attn_prefill if self.kind == "prefill" else m.attn_decode
+            fn(self.cfg, self.batch, self.q, self.caches["k"], self.caches["v"], self.sel, self.out, self.lse,
+               ws[:self.ws_bytes])
         if ev is not None:
             ev[3].record(stream)
 
@@ -121,27 +123,30 @@ class Part:
         return {"bytes": float(cur.sum()) * self.wl.num_kv_heads * 4 + self.sel.numel() * 4}
 
 
-def build_parts(name):
-    """Device inputs of a workload: list of Part (in order) plus total queries."""
+def build_parts(name, batch=None):
+    """Device inputs of a workload: list of Part (in order).  `batch` shrinks
+    a decode workload (fewer sequences, same shapes) for profiling runs."""
     parts = []
-    if name in ("msa_128k_1m", "chunked_prefill_128k"):
+    if name in ("msa_128k_1m", "chunked_prefill_128k", "prefill_128k_last_chunk"):
         chunks = configs.chunked_prefill_128k()
         full = chunks[-1]
         caches = {"k": gen.paged_cache(full, gen.TID_K, device="cuda"),
                   "v": gen.paged_cache(full, gen.TID_V, device="cuda"),
                   "idx_k": gen.paged_cache(full, gen.TID_IDX_K, device="cuda")}
-        out_all = torch.empty((8 * 16384, 64, 128), dtype=torch.bfloat16, device="cuda")
-        for c, wl in enumerate(chunks):
-            parts.append(Part(f"prefill128k/c{c}", wl, caches, "prefill", out_all[c * 16384:(c + 1) * 16384]))
+        which = [7] if name == "prefill_128k_last_chunk" else list(range(8))
+        out_all = torch.empty((len(which) * 16384, 64, 128), dtype=torch.bfloat16, device="cuda")
+        for n, c in enumerate(which):
+            parts.append(Part(f"prefill128k/c{c}", chunks[c], caches, "prefill",
+                              out_all[n * 16384:(n + 1) * 16384]))
     if name in ("msa_128k_1m", "decode_128k", "decode_1m", "verify_ragged"):
         for dn in (("decode_128k", "decode_1m") if name == "msa_128k_1m" else (name,)):
-            wl = configs.ALL[dn]()
+            wl = configs.ALL[dn](batch=batch) if batch else configs.ALL[dn]()
             caches = {"k": gen.paged_cache(wl, gen.TID_K, device="cuda"),
                       "v": gen.paged_cache(wl, gen.TID_V, device="cuda"),
                       "idx_k": gen.paged_cache(wl, gen.TID_IDX_K, device="cuda")}
             parts.append(Part(dn, wl, caches, "decode"))
-    if name in ("prefill_32k", "tiny_prefill_2k"):
-        wl = configs.ALL[name]()
+    if name in ("prefill_32k", "tiny_prefill_2k", "prefill_8k"):
+        wl = configs.prefill_8k() if name == "prefill_8k" else configs.ALL[name]()
         caches = {"k": gen.paged_cache(wl, gen.TID_K, device="cuda"),
                   "v": gen.paged_cache(wl, gen.TID_V, device="cuda"),
                   "idx_k": gen.paged_cache(wl, gen.TID_IDX_K, device="cuda")}
@@ -298,6 +303,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="msa_128k_1m", choices=WORKLOADS)
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--batch", type=int, default=None, help="sequences of a decode workload (profiling)")
+    ap.add_argument("--stop-after", default="attn", choices=("index", "topk", "attn"),
+                    help="profiling: run the step only up to this call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -313,16 +321,16 @@ def main():
     import block_sparse_long_13_b200 as msa
     msa.load_library()  # fails loudly when the CUDA library is missing
 
-    parts = build_parts(args.workload)
+    parts = build_parts(args.workload, args.batch)
     stream = torch.cuda.current_stream()
-    ws_bytes = max(p.ws_bytes for p in parts)
+    ws_bytes = max(p.ws_bytes for p in parts) if args.stop_after == "attn" else 0
     workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     tokens = sum(p.wl.total_q for p in parts)
     nev = len(parts)
 
     def step(evs=None):
         for i, p in enumerate(parts):
-            p.run(workspace, None if evs is None else evs[i], stream)
+            p.run(workspace, None if evs is None else evs[i], stream, args.stop_after)
 
     for _ in range(args.warmup):
         step()

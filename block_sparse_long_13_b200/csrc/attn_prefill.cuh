@@ -27,9 +27,14 @@
 
 namespace msa {
 
-constexpr int ATTP_THREADS = 192;
+constexpr int ATTP_THREADS = 384;  // warpgroup 0: producer + UMMA warps; warpgroups 1, 2: softmax
+// Register split (setmaxnreg): the launch gives 168 per thread (65536 / 384, rounded to 8); warpgroup 0
+// returns registers, the softmax warpgroups take them.  128*56 + 256*224 = 64512 = 384*168.
+constexpr int ATTP_REGS_CTRL = 56, ATTP_REGS_SOFTMAX = 224;
+static_assert(128 * ATTP_REGS_CTRL + 256 * ATTP_REGS_SOFTMAX <= 384 * 168, "register split exceeds the launch");
 constexpr int ATTP_TOK = 8;       // tokens per tile (x 16 heads = 128 MMA rows)
 constexpr int ATTP_G = 16;        // query heads per KV group
+constexpr int ATTP_PHASES = 4;    // tile-list phases walked in lockstep by all CTAs
 constexpr int SCHED_ROWS = 256;   // query rows per schedule CTA
 constexpr int SCHED_SMEM_BUCKETS = 4096;
 
@@ -44,7 +49,9 @@ struct SchedArgs {
   int* cursor;                // [nbuckets]
   int* entries;               // [total_q * Hkv * topk]  (t << 6) | slot
   int* total_tiles;           // [1]
-  int num_seqs, total_q, Hkv, topk, max_blocks, block_size, nbuckets;
+  int4* tile_rec;             // [max_tiles][4]: one 64-byte record per tile
+  const int32_t* page_table;
+  int num_seqs, total_q, Hkv, topk, max_blocks, block_size, nbuckets, num_pages, max_tiles;
 };
 
 __device__ __forceinline__ int entry_bucket(const SchedArgs& a, int t, int g, int b, int s) {
@@ -153,43 +160,63 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(const SchedArgs a) {
   }
 }
 
+// One 64-byte record per tile, so the attention kernel never searches:
+//   int[0] bucket, [1] TMA row of K_b / V_b in the cache = (page * Hkv + g) * 128,
+//   [2] g, [3] b, [4] position offset of the sequence (p = t + off), [5] entries n,
+//   [8 .. 8+n) entries (t << 6 | slot).
+__global__ void __launch_bounds__(256) sched_tiles_kernel(const SchedArgs a) {
+  const int T = min(a.total_tiles[0], a.max_tiles);
+  for (int tile = blockIdx.x * blockDim.x + threadIdx.x; tile < T; tile += gridDim.x * blockDim.x) {
+    int lo = 0, hi = a.nbuckets - 1;  // largest bucket with tile_offsets[bucket] <= tile
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(a.tile_offsets + mid) <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo % a.max_blocks, g = (lo / a.max_blocks) % a.Hkv, seq = lo / (a.max_blocks * a.Hkv);
+    const int e0 = __ldg(a.offsets + lo) + (tile - __ldg(a.tile_offsets + lo)) * ATTP_TOK;
+    const int n = min(ATTP_TOK, __ldg(a.offsets + lo + 1) - e0);
+    int page = __ldg(a.page_table + static_cast<long>(seq) * a.max_blocks + b);
+    if (page < 0 || page >= a.num_pages) { flag_error(MSA_DEV_BOUNDS); page = 0; }
+    const int off = __ldg(a.ctx_len + seq) - __ldg(a.q_start + seq + 1);
+    int ent[ATTP_TOK];
+#pragma unroll
+    for (int e = 0; e < ATTP_TOK; ++e) ent[e] = e < n ? a.entries[e0 + e] : 0;
+    int4* r = a.tile_rec + static_cast<long>(tile) * 4;
+    r[0] = make_int4(lo, (page * a.Hkv + g) * 128, g, b);
+    r[1] = make_int4(off, n, 0, 0);
+    r[2] = make_int4(ent[0], ent[1], ent[2], ent[3]);
+    r[3] = make_int4(ent[4], ent[5], ent[6], ent[7]);
+  }
+}
+
 // ------------------------------------------------------------------ phase 1
 struct AttnPrefillArgs {
-  const int32_t* q_start;
-  const int32_t* ctx_len;
-  const int32_t* page_table;
-  const int* offsets;        // [nbuckets + 1]
-  const int* tile_offsets;   // [nbuckets + 1]
-  const int* entries;
+  const int4* tile_rec;      // [tiles][4] records written by sched_tiles_kernel
   const int* total_tiles;
   float* part_lse;           // [total_q][Hq][topk]
-  int num_seqs, total_q, Hq, Hkv, topk, max_blocks, num_pages, block_size, nbuckets;
+  int Hq, topk, max_tiles;
   float scale_log2;
 };
 
-struct TileInfo {
-  int bucket, seq, g, b, e0, n;  // entries [e0, e0 + n)
+struct TileRec {
+  int bucket, kv_y, g, b, off, n;
+  int ent[ATTP_TOK];
 };
 
-__device__ __forceinline__ void tile_info(const AttnPrefillArgs& a, int tile, TileInfo& ti) {
-  int lo = 0, hi = a.nbuckets - 1;  // largest bucket with tile_offsets[bucket] <= tile
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(a.tile_offsets + mid) <= tile) lo = mid; else hi = mid - 1;
-  }
-  ti.bucket = lo;
-  ti.b = lo % a.max_blocks;
-  ti.g = (lo / a.max_blocks) % a.Hkv;
-  ti.seq = lo / (a.max_blocks * a.Hkv);
-  const int within = tile - __ldg(a.tile_offsets + lo);
-  const int beg = __ldg(a.offsets + lo), end = __ldg(a.offsets + lo + 1);
-  ti.e0 = beg + within * ATTP_TOK;
-  ti.n = min(ATTP_TOK, end - ti.e0);
+__device__ __forceinline__ void load_rec(const int4* base, int tile, TileRec& r) {
+  const int4* p = base + static_cast<long>(tile) * 4;
+  const int4 a = __ldg(p), b = __ldg(p + 1), c = __ldg(p + 2), d = __ldg(p + 3);
+  r.bucket = a.x; r.kv_y = a.y; r.g = a.z; r.b = a.w;
+  r.off = b.x; r.n = b.y;
+  r.ent[0] = c.x; r.ent[1] = c.y; r.ent[2] = c.z; r.ent[3] = c.w;
+  r.ent[4] = d.x; r.ent[5] = d.y; r.ent[6] = d.z; r.ent[7] = d.w;
 }
 
-// shared memory plan (bytes, 1024-aligned): Q[2] 64K | K 32K | V 32K | P[2] 64K | O staging 32K
+// shared memory plan (bytes, 1024-aligned): Q[3] 96K | K 32K | V 32K | P[2] 64K
+// P[w] also stages warpgroup w's O tile for the TMA store once PV has read P.
+constexpr int ATTP_QBUF = 3;      // gathered query tiles in flight (the gather latency needs > 2)
 constexpr int ATTP_QBYTES = 32768, ATTP_KVBYTES = 32768;
-constexpr int ATTP_SMEM = 2 * ATTP_QBYTES + 2 * ATTP_KVBYTES + 2 * 32768 + 32768 + 1024;
+constexpr int ATTP_SMEM = ATTP_QBUF * ATTP_QBYTES + 2 * ATTP_KVBYTES + 2 * 32768 + 1024;
 
 __global__ void __launch_bounds__(ATTP_THREADS, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [total_q*Hq][128]
@@ -199,26 +226,27 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
                     const AttnPrefillArgs a) {
   extern __shared__ __align__(1024) uint8_t dsmem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = smem;                                  // 2 x 32 KiB: [half][128 rows][64]
-  uint8_t* k_s = q_s + 2 * ATTP_QBYTES;                 // [half][128 keys][64]
+  uint8_t* q_s = smem;                                  // 3 x 32 KiB: [half][128 rows][64]
+  uint8_t* k_s = q_s + ATTP_QBUF * ATTP_QBYTES;         // [half][128 keys][64]
   uint8_t* v_s = k_s + ATTP_KVBYTES;                    // [half][128 keys][64]
   uint8_t* p_s = v_s + ATTP_KVBYTES;                    // 2 x 32 KiB: [half][128 rows][64 keys]
-  uint8_t* o_s = p_s + 2 * 32768;                       // [half][128 rows][64]
 
-  __shared__ uint64_t kv_full, kv_empty, q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2],
-      o_full[2], o_empty[2], drain_bar;
+  __shared__ uint64_t kv_full, kv_empty, q_full[ATTP_QBUF], q_empty[ATTP_QBUF], s_full[2], s_empty[2], p_full[2],
+      p_empty[2], o_full[2], o_empty[2], drain_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
-  __shared__ int s_ent[3][ATTP_TOK];   // (t << 6 | slot) of each entry of the last three tiles
+  __shared__ int s_ent[2][2][ATTP_TOK];   // per warpgroup, two tiles: (t << 6 | slot) of each entry
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     s_abort = 0;
     mbar_init(&kv_full, 1);
     mbar_init(&kv_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < ATTP_QBUF; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
       mbar_init(&p_full[i], 4);
@@ -238,11 +266,35 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  const int T = __ldg(a.total_tiles);
-  const int tile0 = static_cast<int>(static_cast<long>(T) * blockIdx.x / gridDim.x);
-  const int tile1 = static_cast<int>(static_cast<long>(T) * (blockIdx.x + 1) / gridDim.x);
-  const int ntile = tile1 - tile0;
+  // The tile list is cut into ATTP_PHASES equal phases (about one KV group each for a
+  // single-sequence prefill); every CTA takes a contiguous share of each phase in turn,
+  // so at any time all CTAs gather query rows of the same phase and those rows stay in L2.
+  const int T = min(__ldg(a.total_tiles), a.max_tiles);
+  static_assert(ATTP_PHASES == 4, "the phase map below is written out for 4 phases");
+  auto share = [&](int q, int& start, int& cnt) {
+    const long p0 = static_cast<long>(T) * q / ATTP_PHASES, p1 = static_cast<long>(T) * (q + 1) / ATTP_PHASES;
+    const long len = p1 - p0;
+    start = static_cast<int>(p0 + len * blockIdx.x / gridDim.x);
+    cnt = static_cast<int>(len * (blockIdx.x + 1) / gridDim.x - len * blockIdx.x / gridDim.x);
+  };
+  int s0, n0, s1, n1, s2, n2, s3, n3;
+  share(0, s0, n0);
+  share(1, s1, n1);
+  share(2, s2, n2);
+  share(3, s3, n3);
+  const int ntile = n0 + n1 + n2 + n3;
+  // global tile of this CTA's i-th tile
+  auto tile_of = [=](int i) -> int {
+    if (i < n0) return s0 + i;
+    i -= n0;
+    if (i < n1) return s1 + i;
+    i -= n1;
+    if (i < n2) return s2 + i;
+    return s3 + (i - n2);
+  };
 
+  if (warp < 4) {
+  regs_dec<ATTP_REGS_CTRL>();
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
     tma_prefetch_desc(&tmap_q);
@@ -250,39 +302,60 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
     tma_prefetch_desc(&tmap_v);
     int cur_bucket = -1;
     uint32_t kvit = 0;
-    int kv_parity = -1, qpar[2] = {-1, -1};
+    int kv_parity = -1;
+    uint32_t q_used = 0, q_parity_bits = 0;   // per query buffer: issued at least once / parity of the last issue
+    TileRec nxt;
+    if (ntile > 0) load_rec(a.tile_rec, tile_of(0), nxt);
     for (int i = 0; i < ntile && !s_abort; ++i) {
-      TileInfo ti;
-      tile_info(a, tile0 + i, ti);
-      if (ti.bucket != cur_bucket) {
+      const TileRec r = nxt;
+      if (i + 1 < ntile) load_rec(a.tile_rec, tile_of(i + 1), nxt);  // in flight while this tile is issued
+      if (r.bucket != cur_bucket) {
         if (!mbar_wait(&kv_empty, (kvit & 1) ^ 1, &s_abort)) break;
-        int page = __ldg(a.page_table + static_cast<long>(ti.seq) * a.max_blocks + ti.b);
-        if (page < 0 || page >= a.num_pages) { flag_error(MSA_DEV_BOUNDS); page = 0; }
-        const int y = (page * a.Hkv + ti.g) * 128;
         mbar_arrive_expect_tx(&kv_full, 2 * ATTP_KVBYTES);
-        tma_load_2d(k_s, &tmap_k, &kv_full, 0, y);
-        tma_load_2d(k_s + 16384, &tmap_k, &kv_full, 64, y);
-        tma_load_2d(v_s, &tmap_v, &kv_full, 0, y);
-        tma_load_2d(v_s + 16384, &tmap_v, &kv_full, 64, y);
+        tma_load_2d(k_s, &tmap_k, &kv_full, 0, r.kv_y);
+        tma_load_2d(k_s + 16384, &tmap_k, &kv_full, 64, r.kv_y);
+        tma_load_2d(v_s, &tmap_v, &kv_full, 0, r.kv_y);
+        tma_load_2d(v_s + 16384, &tmap_v, &kv_full, 64, r.kv_y);
         kv_parity = kvit & 1;
         ++kvit;
-        cur_bucket = ti.bucket;
+        cur_bucket = r.bucket;
       }
-      const int qb = i & 1;
-      if (!mbar_wait(&q_empty[qb], ((i >> 1) & 1) ^ 1, &s_abort)) break;
-      mbar_arrive_expect_tx(&q_full[qb], ti.n * 4096);
-      for (int e = 0; e < ti.n; ++e) {
-        const int ent = __ldg(a.entries + ti.e0 + e);
-        const int t = ent >> 6;
-        const int y = t * a.Hq + ti.g * ATTP_G;
-        tma_load_2d(q_s + qb * ATTP_QBYTES + e * 2048, &tmap_q, &q_full[qb], 0, y);
-        tma_load_2d(q_s + qb * ATTP_QBYTES + 16384 + e * 2048, &tmap_q, &q_full[qb], 64, y);
+      const int qb = i % ATTP_QBUF;
+      const uint32_t qpar = static_cast<uint32_t>((i / ATTP_QBUF) & 1);
+      if (!mbar_wait(&q_empty[qb], qpar ^ 1u, &s_abort)) break;
+      mbar_arrive_expect_tx(&q_full[qb], r.n * 4096);
+#pragma unroll
+      for (int e = 0; e < ATTP_TOK; ++e) {
+        if (e < r.n) {
+          const int y = (r.ent[e] >> 6) * a.Hq + r.g * ATTP_G;
+          tma_load_2d(q_s + qb * ATTP_QBYTES + e * 2048, &tmap_q, &q_full[qb], 0, y);
+          tma_load_2d(q_s + qb * ATTP_QBYTES + 16384 + e * 2048, &tmap_q, &q_full[qb], 64, y);
+        }
       }
-      qpar[qb] = (i >> 1) & 1;
+      q_used |= 1u << qb;
+      q_parity_bits = (q_parity_bits & ~(1u << qb)) | (qpar << qb);
+      // warm L2 with the next tile's query rows (and its K/V when the bucket changes)
+      if (i + 1 < ntile) {
+#pragma unroll
+        for (int e = 0; e < ATTP_TOK; ++e) {
+          if (e < nxt.n) {
+            const int y = (nxt.ent[e] >> 6) * a.Hq + nxt.g * ATTP_G;
+            tma_prefetch_l2_2d(&tmap_q, 0, y);
+            tma_prefetch_l2_2d(&tmap_q, 64, y);
+          }
+        }
+        if (nxt.bucket != r.bucket) {
+          tma_prefetch_l2_2d(&tmap_k, 0, nxt.kv_y);
+          tma_prefetch_l2_2d(&tmap_k, 64, nxt.kv_y);
+          tma_prefetch_l2_2d(&tmap_v, 0, nxt.kv_y);
+          tma_prefetch_l2_2d(&tmap_v, 64, nxt.kv_y);
+        }
+      }
     }
     if (s_abort) {
       if (kv_parity >= 0) mbar_wait_drain(&kv_full, kv_parity);
-      for (int j = 0; j < 2; ++j) if (qpar[j] >= 0) mbar_wait_drain(&q_full[j], qpar[j]);
+      for (int j = 0; j < ATTP_QBUF; ++j)
+        if (q_used & (1u << j)) mbar_wait_drain(&q_full[j], (q_parity_bits >> j) & 1u);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ UMMA issuer
@@ -305,14 +378,14 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
         umma_bf16_ss(d, adesc, bdesc, id_pv, kk > 0 ? 1u : 0u);
       }
       umma_commit(&o_full[pb]);
-      umma_commit(&p_empty[pb]);
       return true;
     };
     bool ok = true;
+    int nbucket = ntile > 0 ? __ldg(&a.tile_rec[static_cast<long>(tile_of(0)) * 4].x) : -1;
     for (int i = 0; i < ntile && ok && !s_abort; ++i) {
-      TileInfo ti;
-      tile_info(a, tile0 + i, ti);
-      if (ti.bucket != cur_bucket) {
+      const int bucket = nbucket;
+      if (i + 1 < ntile) nbucket = __ldg(&a.tile_rec[static_cast<long>(tile_of(i + 1)) * 4].x);
+      if (bucket != cur_bucket) {
         if (pv_pending) {  // finish the previous bucket before its K/V is replaced
           if (!issue_pv(i - 1)) break;
           pv_pending = false;
@@ -320,20 +393,20 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
         if (cur_bucket >= 0) umma_commit(&kv_empty);
         if (!mbar_wait(&kv_full, kvit & 1, &s_abort)) break;
         ++kvit;
-        cur_bucket = ti.bucket;
+        cur_bucket = bucket;
       }
-      const int qb = i & 1;
-      if (!mbar_wait(&q_full[qb], (i >> 1) & 1, &s_abort)) break;
-      if (!mbar_wait(&s_empty[qb], ((i >> 1) & 1) ^ 1, &s_abort)) break;
+      const int qb = i % ATTP_QBUF, sb = i & 1;
+      if (!mbar_wait(&q_full[qb], (i / ATTP_QBUF) & 1, &s_abort)) break;
+      if (!mbar_wait(&s_empty[sb], ((i >> 1) & 1) ^ 1, &s_abort)) break;
       tc_fence_after();
-      const uint32_t d = tmem + qb * 128;
+      const uint32_t d = tmem + sb * 128;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
         umma_bf16_ss(d, sdesc_sw128(qa + qb * ATTP_QBYTES + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), id_s,
                      kk > 0 ? 1u : 0u);
       }
-      umma_commit(&s_full[qb]);
+      umma_commit(&s_full[sb]);
       umma_commit(&q_empty[qb]);
       if (pv_pending) ok = issue_pv(i - 1);
       pv_pending = true;
@@ -343,125 +416,141 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0);
     }
-  } else if (warp >= 2) {
-    // ------------------------------------------------------------ softmax + epilogue
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;           // MMA row = entry * 16 + head
+  }
+  } else {
+    regs_inc<ATTP_REGS_SOFTMAX>();
+    // ------------------------------------------------------------ two softmax + epilogue warpgroups
+    // warpgroup w takes the CTA's tiles i = w, w + 2, ...; it owns Q/S/P/O buffers w
+    const int w = (warp - 4) >> 2;
+    const int bar = 1 + w;                        // named barrier of this warpgroup
+    const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;            // MMA row = entry * 16 + head
     const int e = r >> 4, h = r & 15;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const bool issuer = (warp == 2 && lane == 0);
+    const bool issuer = (warp == 4 + 4 * w && lane == 0);
     const float LN2 = 0.69314718055994531f;
-    // the previous tile's row state, consumed by its deferred epilogue
-    int pv_t = 0, pv_slot = 0, pv_g = 0, pv_n = 0;
-    bool pv_valid = false;
-    float pv_m = 0.f, pv_l = 1.f;
+    const float sc = a.scale_log2;
+    const uint64_t pol_stream = l2_policy_evict_first();
+    uint8_t* pbuf = p_s + w * 32768;
+    const int nj = (ntile - w + 1) / 2;
+    // the fields this row needs of its tiles, prefetched one tile ahead
+    struct RowRec { int g, b, off, n, ent; };
+    auto load_row = [&](int tile) -> RowRec {
+      const int4* p = a.tile_rec + static_cast<long>(tile) * 4;
+      const int4 h0 = __ldg(p);
+      const int4 h1 = __ldg(p + 1);
+      RowRec rr;
+      rr.g = h0.z; rr.b = h0.w; rr.off = h1.x; rr.n = h1.y;
+      rr.ent = __ldg(reinterpret_cast<const int*>(p + 2) + e);
+      return rr;
+    };
+    RowRec nxt{};
+    if (nj > 0) nxt = load_row(tile_of(w));
+    for (int j = 0; j < nj; ++j) {               // every exit decision is uniform over the warpgroup
+      const int i = 2 * j + w;
+      const RowRec rec = nxt;
+      if (j + 1 < nj) nxt = load_row(tile_of(i + 2));
+      const bool valid = e < rec.n;
+      const int ent = rec.ent;
+      const int t = ent >> 6, slot = ent & 63;
+      const int vis = valid ? min(128, t + rec.off - rec.b * 128 + 1) : 128;  // visible keys of the block
+      if (valid && h == 0) s_ent[w][j & 1][e] = ent;
+      const uint32_t par = static_cast<uint32_t>(j & 1);
 
-    // store tile j's O / l (bf16) through the staging tile with TMA, and its lse
-    auto epilogue = [&](int j) -> bool {
-      const int ob = j & 1;
-      if (!mbar_wait_group(&o_full[ob], (j >> 1) & 1, &s_abort, 2, 128)) return false;
+      // ---- S = Q K^T is in TMEM: the row's 128 scores in registers, max over the visible keys
+      if (!mbar_wait_group(&s_full[w], par, &s_abort, bar, 128)) break;
       tc_fence_after();
-      if (issuer) bulk_wait_read_all();          // the staging tile has been read by earlier stores
-      named_bar_sync(1, 128);
-      const float inv = 1.f / pv_l;
+      const uint32_t s_addr = lane_addr + w * 128;
+      float v0[32], v1[32], v2[32], v3[32];
+      tmem_ld32(s_addr, v0);
+      tmem_ld32(s_addr + 32, v1);
+      tmem_ld32(s_addr + 64, v2);
+      tmem_ld32(s_addr + 96, v3);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[w]);    // S[w] has been read
+      if (vis < 128) {                            // the query's own block: keys after it do not count
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (c >= vis) v0[c] = -INFINITY;
+          if (32 + c >= vis) v1[c] = -INFINITY;
+          if (64 + c >= vis) v2[c] = -INFINITY;
+          if (96 + c >= vis) v3[c] = -INFINITY;
+        }
+      }
+      float mx[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) mx[c & 7] = fmax3(mx[c & 7], fmaxf(v0[c], v1[c]), fmaxf(v2[c], v3[c]));
+      const float m = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], fmax3(mx[4], mx[5], mx[6]), mx[7]));
+      const float mc = (m > -INFINITY) ? m * sc : 0.f;   // -inf only on rows past the tile's entries
+      // ---- P = exp2(scale * S - max) as bf16 into P[w] (free once the last stores from it were read)
+      if (issuer) bulk_wait_read_all();
+      named_bar_sync(bar, 128);
+      float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+      for (int q8 = 0; q8 < 16; ++q8) {
+        float pe[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int c = q8 * 8 + u;
+          const float x = c < 32 ? v0[c] : c < 64 ? v1[c - 32] : c < 96 ? v2[c - 64] : v3[c - 96];
+          pe[u] = exp2f(fmaf(x, sc, -mc));        // exp2(-inf) = 0 for masked keys
+        }
+        l0 += (pe[0] + pe[1]) + (pe[2] + pe[3]);
+        l1 += (pe[4] + pe[5]) + (pe[6] + pe[7]);
+        uint4 wv;
+        wv.x = pack_bf16(pe[0], pe[1]);
+        wv.y = pack_bf16(pe[2], pe[3]);
+        wv.z = pack_bf16(pe[4], pe[5]);
+        wv.w = pack_bf16(pe[6], pe[7]);
+        *reinterpret_cast<uint4*>(pbuf + (q8 >> 3) * 16384 + sw128_offset(r, (q8 & 7) * 16)) = wv;
+      }
+      const float l = l0 + l1;
+      fence_proxy_async_smem();                   // P visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[w]);
+
+      // ---- O = P V is in TMEM: O / l as bf16, staged in P[w] for the TMA store
+      if (!mbar_wait_group(&o_full[w], par, &s_abort, bar, 128)) break;
+      tc_fence_after();
+      const float inv = 1.f / l;
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         float v[32];
-        tmem_ld32(lane_addr + 256 + ob * 128 + c4 * 32, v);
+        tmem_ld32(lane_addr + 256 + w * 128 + c4 * 32, v);
         tmem_ld_wait();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          const int col = c4 * 32 + q8 * 8;      // output dims col .. col+7
-          uint4 w;
-          w.x = pack_bf16(v[q8 * 8 + 0] * inv, v[q8 * 8 + 1] * inv);
-          w.y = pack_bf16(v[q8 * 8 + 2] * inv, v[q8 * 8 + 3] * inv);
-          w.z = pack_bf16(v[q8 * 8 + 4] * inv, v[q8 * 8 + 5] * inv);
-          w.w = pack_bf16(v[q8 * 8 + 6] * inv, v[q8 * 8 + 7] * inv);
-          *reinterpret_cast<uint4*>(o_s + (col >> 6) * 16384 + sw128_offset(r, (col & 63) * 2)) = w;
+          const int col = c4 * 32 + q8 * 8;       // output dims col .. col+7
+          uint4 wv;
+          wv.x = pack_bf16(v[q8 * 8 + 0] * inv, v[q8 * 8 + 1] * inv);
+          wv.y = pack_bf16(v[q8 * 8 + 2] * inv, v[q8 * 8 + 3] * inv);
+          wv.z = pack_bf16(v[q8 * 8 + 4] * inv, v[q8 * 8 + 5] * inv);
+          wv.w = pack_bf16(v[q8 * 8 + 6] * inv, v[q8 * 8 + 7] * inv);
+          *reinterpret_cast<uint4*>(pbuf + (col >> 6) * 16384 + sw128_offset(r, (col & 63) * 2)) = wv;
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[ob]);
-      if (pv_valid)
-        a.part_lse[(static_cast<long>(pv_t) * a.Hq + pv_g * ATTP_G + h) * a.topk + pv_slot] =
-            (pv_m + log2f(pv_l)) * LN2;
+      if (lane == 0) mbar_arrive(&o_empty[w]);
+      if (valid)
+        a.part_lse[(static_cast<long>(t) * a.Hq + rec.g * ATTP_G + h) * a.topk + slot] = (mc + log2f(l)) * LN2;
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
+      named_bar_sync(bar, 128);
       if (issuer) {
-        for (int ee = 0; ee < pv_n; ++ee) {
-          const int ent = s_ent[j % 3][ee];
-          const int y = ((ent >> 6) * a.topk + (ent & 63)) * a.Hq + pv_g * ATTP_G;
-          tma_store_2d(&tmap_po, o_s + ee * 2048, 0, y);
-          tma_store_2d(&tmap_po, o_s + 16384 + ee * 2048, 64, y);
+        for (int ee = 0; ee < rec.n; ++ee) {
+          const int en = s_ent[w][j & 1][ee];
+          const int y = ((en >> 6) * a.topk + (en & 63)) * a.Hq + rec.g * ATTP_G;
+          tma_store_2d_hint(&tmap_po, pbuf + ee * 2048, 0, y, pol_stream);
+          tma_store_2d_hint(&tmap_po, pbuf + 16384 + ee * 2048, 64, y, pol_stream);
         }
         bulk_commit();
       }
-      return true;
-    };
-
-    bool ok = true;
-    for (int i = 0; i < ntile && ok; ++i) {   // every exit decision is uniform over the group
-      TileInfo ti;
-      tile_info(a, tile0 + i, ti);
-      const int sb = i & 1;
-      const bool valid = e < ti.n;
-      int t = 0, slot = 0, p = 0;
-      if (valid) {
-        const int ent = __ldg(a.entries + ti.e0 + e);
-        t = ent >> 6;
-        slot = ent & 63;
-        const int qs = __ldg(a.q_start + ti.seq), nq = __ldg(a.q_start + ti.seq + 1) - qs;
-        p = __ldg(a.ctx_len + ti.seq) - nq + (t - qs);
-        if (h == 0) s_ent[i % 3][e] = ent;
-      }
-      const int vis = valid ? min(128, p - ti.b * a.block_size + 1) : 128;
-      // ---- softmax of tile i: scale, mask keys after the query, exp2, row sum
-      if (!mbar_wait_group(&s_full[sb], (i >> 1) & 1, &s_abort, 2, 128)) { ok = false; break; }
-      tc_fence_after();
-      float sv[128];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float tmp[32];
-        tmem_ld32(lane_addr + sb * 128 + c4 * 32, tmp);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) sv[c4 * 32 + c] = tmp[c];
-      }
-      tmem_ld_wait();
-      float m = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        sv[c] = (c < vis) ? sv[c] * a.scale_log2 : -INFINITY;
-        m = fmaxf(m, sv[c]);
-      }
-      if (!(m > -INFINITY)) m = 0.f;             // only rows past the tile's entries
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);  // S[sb] has been read
-      if (!mbar_wait_group(&p_empty[sb], ((i >> 1) & 1) ^ 1, &s_abort, 2, 128)) { ok = false; break; }
-      float l = 0.f;
-      uint8_t* pbuf = p_s + sb * 32768;
-#pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        float pe[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) { pe[u] = exp2f(sv[c8 * 8 + u] - m); l += pe[u]; }
-        uint4 w;
-        w.x = pack_bf16(pe[0], pe[1]);
-        w.y = pack_bf16(pe[2], pe[3]);
-        w.z = pack_bf16(pe[4], pe[5]);
-        w.w = pack_bf16(pe[6], pe[7]);
-        *reinterpret_cast<uint4*>(pbuf + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16)) = w;
-      }
-      fence_proxy_async_smem();                  // P visible to the tensor core
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
-      // ---- deferred epilogue of tile i-1 (its PV overlapped this softmax)
-      if (i > 0 && !epilogue(i - 1)) { ok = false; break; }
-      pv_t = t; pv_slot = slot; pv_g = ti.g; pv_n = ti.n; pv_valid = valid; pv_m = m; pv_l = l;
     }
-    if (ok && ntile > 0) epilogue(ntile - 1);
-    if (issuer) bulk_wait_all();                 // partial stores complete before exit
+    if (issuer) bulk_wait_all();                  // partial stores complete before exit
   }
   __syncwarp();
   tc_fence_before();

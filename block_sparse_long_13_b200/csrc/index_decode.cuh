@@ -11,22 +11,25 @@
 //
 // The pass is HBM-bound: every indexer key of every visible page is read
 // once.  Persistent CTAs (one per SM) own contiguous runs of (sequence,
-// page) units; each unit is read as H_kv TMA tiles of hg x 128 x 64 bf16
-// (hg = indexer heads per group, 128-byte swizzle) through a STAGES-deep
-// ring of shared-memory buffers.  Each thread owns one key row, widens it to
-// fp32 and dots it with the sequence's (<= 8) queries held in shared memory;
-// the block max is a warp redux.sync on order-preserving integer keys.
+// page) units.  Warp 0 is the producer: it reads the page ids of 32 units at
+// a time (one coalesced load) and streams each unit as H_kv TMA tiles of
+// hg x 128 x 64 bf16 (128-byte swizzle) through a ring of shared buffers
+// guarded by full/empty mbarriers.  Warps 1..8 consume: each thread owns one
+// key row, widens it to fp32 and dots it with the sequence's (<= 8) queries
+// held in shared memory; the block max is a warp redux.sync on
+// order-preserving integer keys, then a per-group sum over the heads.
 #pragma once
 #include "common.cuh"
 
 namespace msa {
 
-constexpr int IDXD_THREADS = 256;
+constexpr int IDXD_CONSUMERS = 256;
+constexpr int IDXD_THREADS = 32 + IDXD_CONSUMERS;
 constexpr int IDXD_MAXQ = 8;       // queries per sequence handled by this form
 constexpr int IDXD_MAXHG = 8;      // indexer heads per KV group
 constexpr int IDXD_MAXHI = 16;     // indexer heads
 constexpr int IDXD_MAXSEQ = 2048;  // sequences per call for this form
-constexpr int IDXD_RING_BYTES = 160 * 1024;
+constexpr int IDXD_SMEM_BUDGET = 212 * 1024;  // dynamic: key ring + this call's queries
 
 struct IdxDecodeArgs {
   const __nv_bfloat16* idx_q;   // [total_q][Hi][64]
@@ -38,20 +41,21 @@ struct IdxDecodeArgs {
   int stage_bytes, stages;
 };
 
+// NQ: compile-time bound on the queries of any sequence (1, 2, 4 or 8)
+template <int NQ>
 __global__ void __launch_bounds__(IDXD_THREADS, 1)
 index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t dsmem[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full_bar[16];
+  __shared__ uint64_t full_bar[16], empty_bar[16];
   __shared__ int s_nbprefix[IDXD_MAXSEQ + 1];
-  __shared__ __align__(16) float s_q[IDXD_MAXQ * IDXD_MAXHI * 64];  // current sequence: queries of all heads (fp32)
-  __shared__ uint32_t s_part[2][IDXD_MAXQ][IDXD_MAXHG][4];
+  __shared__ uint32_t s_part[2][NQ][IDXD_MAXHG][4];
+  // current sequence's queries of all heads, fp32, after the key ring
+  float* s_q = reinterpret_cast<float*>(ring + static_cast<long>(a.stages) * a.stage_bytes);
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int token = tid & 127;
-  const int hl0 = tid >> 7;  // 0 or 1
 
   // blocks per sequence (0 for sequences without queries), prefix in smem
   if (tid == 0) {
@@ -66,7 +70,10 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
       acc += nb;
       s_nbprefix[s + 1] = acc;
     }
-    for (int i = 0; i < a.stages; ++i) mbar_init(&full_bar[i], 1);
+    for (int i = 0; i < a.stages; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], IDXD_CONSUMERS / 32);
+    }
     fence_mbar_init();
   }
   __syncthreads();
@@ -74,9 +81,9 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
   const long u0 = total_units * blockIdx.x / gridDim.x;
   const long u1 = total_units * (blockIdx.x + 1) / gridDim.x;
   const long nstage = (u1 - u0) * a.Hkv;
-  if (nstage == 0) return;
+  if (nstage == 0) return;  // uniform
 
-  // unit -> (seq, block): seq-major walk
+  // unit -> (seq, block): seq-major order
   auto locate = [&](long u, int& s, int& b) {
     int lo = 0, hi = a.num_seqs - 1;
     while (lo < hi) {  // largest s with prefix[s] <= u
@@ -87,100 +94,134 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
     b = static_cast<int>(u - s_nbprefix[lo]);
   };
 
-  // producer state (thread 0): issue stage k into slot k % stages
-  auto issue = [&](long k) {
-    const long u = u0 + k / a.Hkv;
-    const int g = static_cast<int>(k % a.Hkv);
-    int s, b;
-    locate(u, s, b);
-    int page = __ldg(a.page_table + static_cast<long>(s) * a.max_blocks + b);
-    if (page < 0 || page >= a.num_pages) { flag_error(MSA_DEV_BOUNDS); page = 0; }
-    const int slot = static_cast<int>(k % a.stages);
-    mbar_arrive_expect_tx(&full_bar[slot], a.stage_bytes);
-    tma_load_4d(ring + static_cast<long>(slot) * a.stage_bytes, &tmap_k, &full_bar[slot], 0, 0, g * a.hg, page);
-  };
-  long issued = 0, kstop = -1;
-  if (tid == 0) {
-    tma_prefetch_desc(&tmap_k);
-    for (long k = 0; k < nstage && k < a.stages; ++k) { issue(k); ++issued; }
-  }
-
-  int cur_seq = -1, nq = 0, qrow0 = 0, ctx = 0;
-  for (long k = 0; k < nstage; ++k) {
-    const long u = u0 + k / a.Hkv;
-    const int g = static_cast<int>(k % a.Hkv);
-    int s, b;
-    locate(u, s, b);
-    if (s != cur_seq) {
-      // load this sequence's queries (all indexer heads) as fp32
-      __syncthreads();
-      cur_seq = s;
-      qrow0 = __ldg(a.q_start + s);
-      nq = __ldg(a.q_start + s + 1) - qrow0;
-      ctx = __ldg(a.ctx_len + s);
-      if (nq > IDXD_MAXQ) { if (tid == 0) flag_error(MSA_DEV_BOUNDS); nq = IDXD_MAXQ; }
-      const int n = nq * a.Hi * 64;
-      const __nv_bfloat16* src = a.idx_q + static_cast<long>(qrow0) * a.Hi * 64;
-      for (int i = tid; i < n; i += IDXD_THREADS) s_q[i] = __bfloat162float(src[i]);
-      __syncthreads();
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer warp
+    if (lane == 0) tma_prefetch_desc(&tmap_k);
+    int page_l = 0;
+    uint32_t used = 0, parity_bits = 0;   // per ring slot: issued at least once / parity of the last issue
+    for (long k = 0; k < nstage; ++k) {
+      const long j = k / a.Hkv;           // unit index within this CTA
+      const int g = static_cast<int>(k % a.Hkv);
+      if (g == 0 && (j & 31) == 0) {      // page ids of the next 32 units, one per lane
+        const long uu = u0 + j + lane;
+        page_l = 0;
+        if (uu < u1) {
+          int s, b;
+          locate(uu, s, b);
+          page_l = __ldg(a.page_table + static_cast<long>(s) * a.max_blocks + b);
+          if (page_l < 0 || page_l >= a.num_pages) { flag_error(MSA_DEV_BOUNDS); page_l = 0; }
+        }
+      }
+      const int page = __shfl_sync(0xFFFFFFFFu, page_l, static_cast<int>(j & 31));
+      const int slot = static_cast<int>(k % a.stages);
+      const uint32_t par = static_cast<uint32_t>((k / a.stages) & 1);
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(&empty_bar[slot], par ^ 1u, &s_abort);
+        if (ok) {
+          mbar_arrive_expect_tx(&full_bar[slot], a.stage_bytes);
+          tma_load_4d(ring + static_cast<long>(slot) * a.stage_bytes, &tmap_k, &full_bar[slot], 0, 0, g * a.hg,
+                      page);
+          used |= 1u << slot;
+          parity_bits = (parity_bits & ~(1u << slot)) | (par << slot);
+        }
+      }
+      if (__any_sync(0xFFFFFFFFu, !ok)) break;
     }
-    const int slot = static_cast<int>(k % a.stages);
-    const uint32_t parity = static_cast<uint32_t>((k / a.stages) & 1);
-    const bool ok = mbar_wait(&full_bar[slot], parity, &s_abort);
-    const uint8_t* tile = ring + static_cast<long>(slot) * a.stage_bytes;
-    const int j = b * a.block_size + token;  // absolute key position
-    const int pbuf = static_cast<int>(k & 1);
-    for (int hl = hl0; ok && hl < a.hg; hl += 2) {
-      // this thread's key row: 64 bf16, 128-byte swizzled
-      const uint8_t* rowp = tile + (hl * 128 + token) * 128;
-      float acc[IDXD_MAXQ];
+    if (lane == 0 && s_abort) {  // let issued copies land before the CTA exits
+      for (int i = 0; i < a.stages; ++i)
+        if (used & (1u << i)) mbar_wait_drain(&full_bar[i], (parity_bits >> i) & 1u);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int c = tid - 32;
+    const int cw = c >> 5;               // consumer warp 0..7
+    const int token = c & 127;
+    const int hl0 = c >> 7;              // 0 or 1
+    int cur_seq = -1, nq = 0, qrow0 = 0, ctx = 0;
+    int s, b;
+    locate(u0, s, b);
+    // the per-group sum of stage k-1 is made after the barrier that opens stage k
+    int pv_nq = 0, pv_row0 = 0, pv_g = 0, pv_b = 0;
+    auto combine = [&](int pbuf) {
+      if (c < pv_nq) {
+        float tot = 0.f;
+        for (int hl = 0; hl < a.hg; ++hl) {
+          const uint32_t* pp = s_part[pbuf][c][hl];
+          tot += key_to_float(max(max(pp[0], pp[1]), max(pp[2], pp[3])));
+        }
+        a.scores[(static_cast<long>(pv_row0 + c) * a.Hkv + pv_g) * a.max_blocks + pv_b] = tot;
+      }
+    };
+    bool ok = true;
+    for (long k = 0; k < nstage; ++k) {
+      const int g = static_cast<int>(k % a.Hkv);
+      if (k > 0 && g == 0) {  // next unit: next block, or the next sequence with blocks
+        ++b;
+        while (b >= s_nbprefix[s + 1] - s_nbprefix[s]) { ++s; b = 0; }
+      }
+      if (s != cur_seq) {
+        // this sequence's queries (all indexer heads) as fp32
+        named_bar_sync(1, IDXD_CONSUMERS);
+        cur_seq = s;
+        qrow0 = __ldg(a.q_start + s);
+        nq = __ldg(a.q_start + s + 1) - qrow0;
+        ctx = __ldg(a.ctx_len + s);
+        if (nq > NQ) { if (c == 0) flag_error(MSA_DEV_BOUNDS); nq = NQ; }
+        const int n = nq * a.Hi * 64;
+        const __nv_bfloat16* src = a.idx_q + static_cast<long>(qrow0) * a.Hi * 64;
+        for (int i = c; i < n; i += IDXD_CONSUMERS) s_q[i] = __bfloat162float(src[i]);
+        named_bar_sync(1, IDXD_CONSUMERS);
+      }
+      const int slot = static_cast<int>(k % a.stages);
+      const uint32_t par = static_cast<uint32_t>((k / a.stages) & 1);
+      if (!mbar_wait_group(&full_bar[slot], par, &s_abort, 2, IDXD_CONSUMERS)) { ok = false; break; }
+      if (k > 0) combine(static_cast<int>((k - 1) & 1));
+      const uint8_t* tile = ring + static_cast<long>(slot) * a.stage_bytes;
+      const int j = b * a.block_size + token;  // absolute key position
+      const int pbuf = static_cast<int>(k & 1);
+      for (int hl = hl0; hl < a.hg; hl += 2) {
+        // this thread's key row: 64 bf16, 128-byte swizzled
+        const uint8_t* rowp = tile + (hl * 128 + token) * 128;
+        float ac0[NQ], ac1[NQ];
 #pragma unroll
-      for (int i = 0; i < IDXD_MAXQ; ++i) acc[i] = 0.f;
-      const int h = g * a.hg + hl;
+        for (int i = 0; i < NQ; ++i) { ac0[i] = 0.f; ac1[i] = 0.f; }
+        const int h = g * a.hg + hl;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((c ^ (token & 7)) << 4));
-        const float kf[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
-                             bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((cc ^ (token & 7)) << 4));
+          const float kf[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
+                               bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
 #pragma unroll
-        for (int i = 0; i < IDXD_MAXQ; ++i) {
-          if (i < nq) {
-            const float4* qp = reinterpret_cast<const float4*>(s_q + (i * a.Hi + h) * 64 + c * 8);
-            const float4 q0 = qp[0], q1 = qp[1];
-            float t = acc[i];
-            t = fmaf(q0.x, kf[0], t); t = fmaf(q0.y, kf[1], t); t = fmaf(q0.z, kf[2], t); t = fmaf(q0.w, kf[3], t);
-            t = fmaf(q1.x, kf[4], t); t = fmaf(q1.y, kf[5], t); t = fmaf(q1.z, kf[6], t); t = fmaf(q1.w, kf[7], t);
-            acc[i] = t;
+          for (int i = 0; i < NQ; ++i) {
+            if (NQ == 1 || i < nq) {
+              const float4* qp = reinterpret_cast<const float4*>(s_q + (i * a.Hi + h) * 64 + cc * 8);
+              const float4 q0 = qp[0], q1 = qp[1];
+              float t0 = ac0[i], t1 = ac1[i];
+              t0 = fmaf(q0.x, kf[0], t0); t1 = fmaf(q0.y, kf[1], t1); t0 = fmaf(q0.z, kf[2], t0); t1 = fmaf(q0.w, kf[3], t1);
+              t0 = fmaf(q1.x, kf[4], t0); t1 = fmaf(q1.y, kf[5], t1); t0 = fmaf(q1.z, kf[6], t0); t1 = fmaf(q1.w, kf[7], t1);
+              ac0[i] = t0; ac1[i] = t1;
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+          if (NQ == 1 || i < nq) {
+            const int p = ctx - nq + i;
+            const float v = (j <= p) ? ac0[i] + ac1[i] : -INFINITY;
+            const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, order_key(v));
+            if (lane == 0) s_part[pbuf][i][hl][cw & 3] = m;
           }
         }
       }
-#pragma unroll
-      for (int i = 0; i < IDXD_MAXQ; ++i) {
-        if (i < nq) {
-          const int p = ctx - nq + i;
-          const float v = (j <= p) ? acc[i] : -INFINITY;
-          const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, order_key(v));
-          if (lane == 0) s_part[pbuf][i][hl][warp & 3] = m;
-        }
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[slot]);  // this warp is done with the tile
+      pv_nq = nq; pv_row0 = qrow0; pv_g = g; pv_b = b;
     }
-    __syncthreads();  // slot consumed, partial maxima visible, abort flag uniform
-    if (s_abort) { kstop = k; break; }
-    if (tid == 0 && k + a.stages < nstage) { issue(k + a.stages); ++issued; }
-    if (tid < nq) {
-      float tot = 0.f;
-      for (int hl = 0; hl < a.hg; ++hl) {
-        const uint32_t* pp = s_part[pbuf][tid][hl];
-        const uint32_t m = max(max(pp[0], pp[1]), max(pp[2], pp[3]));
-        tot += key_to_float(m);
-      }
-      a.scores[(static_cast<long>(qrow0 + tid) * a.Hkv + g) * a.max_blocks + b] = tot;
+    if (ok && nstage > 0) {
+      named_bar_sync(1, IDXD_CONSUMERS);               // last stage's partial maxima visible
+      combine(static_cast<int>((nstage - 1) & 1));
     }
-  }
-  // after a timeout, let the copies still in flight land (bounded) before the CTA exits
-  if (tid == 0 && kstop >= 0) {
-    for (long kk = kstop; kk < issued; ++kk)
-      mbar_wait_drain(&full_bar[kk % a.stages], static_cast<uint32_t>((kk / a.stages) & 1));
   }
 }
 

@@ -5,27 +5,30 @@
 // (inteligile "MiniMax-M3" model page, row "Indexer-selected sparse
 // attention"; 24-ai.news, block scoring per query group).
 //
-// Work unit = (sequence, tile of 128 query rows, KV group g).  For each
-// causally visible key block b the unit computes, per indexer head of the
-// group, the 128 x 128 score tile Q_h K_h^T (K = 64) with tcgen05.mma into a
-// TMEM accumulator, and four epilogue warps (thread = query row = TMEM lane)
-// max-pool the row over the block's visible keys and sum over the heads.
+// Work unit = (sequence, tile of 128 query rows, KV group g).  The unit walks
+// its causally visible key blocks in pairs; one step = (block pair, indexer
+// head h of the group): a single 128 x 256 x 64 product Q_h [K_h(b) ; K_h(b+1)]^T
+// on tcgen05 into a 256-column TMEM accumulator (N = 256 keeps the 1-SM tensor
+// core at full rate; N = 128 runs it at half rate).  Two epilogue warpgroups
+// read every step, one block of the pair each (thread = query row = TMEM
+// lane), max-pool the row over the block's visible keys and sum the group's
+// heads in registers before writing the block score.
 //
-// Roles: warp 0 = TMA producer (query tile once per unit, key tiles through a
-// STAGES-deep ring), warp 1 = TMEM owner + single-thread UMMA issuer, warps
-// 2..5 = epilogue.  Accumulators are double-buffered in TMEM (4 / hg
-// buffers of hg x 128 fp32 columns) so the tensor core computes block b+1
-// while the epilogue pools block b.  Units are dealt to persistent CTAs in
-// snake order over a longest-first list (a query tile's cost grows with its
-// position).
+// Roles: warp 0 = TMA producer (query tiles double-buffered, key tiles of a
+// (pair, head) through a ring), warp 1 = TMEM owner + single-thread UMMA
+// issuer, warps 2..5 / 6..9 = the two epilogue warpgroups.  Accumulators are
+// double-buffered (2 x 256 columns).  Units are dealt to persistent CTAs in a
+// snake order over a longest-first list, group-major so that one group's keys
+// are live in L2 at a time.
 #pragma once
 #include "common.cuh"
 
 namespace msa {
 
-constexpr int IDXP_THREADS = 192;
+constexpr int IDXP_THREADS = 320;
 constexpr int IDXP_TILE = 128;
 constexpr int IDXP_MAXSEQ = 1024;
+constexpr int IDXP_STAGE_BYTES = 2 * IDXP_TILE * 64 * 2;   // keys of one head for two blocks: 32 KiB
 
 struct IdxPrefillArgs {
   float* scores;             // [total_q][Hkv][max_blocks]
@@ -33,7 +36,7 @@ struct IdxPrefillArgs {
   const int32_t* ctx_len;
   const int32_t* page_table;
   int num_seqs, total_q, max_blocks, num_pages, Hi, Hkv, hg, block_size;
-  int stages, nbuf;          // K ring depth; TMEM accumulator buffers
+  int stages, nqbuf;         // key ring depth; query tile buffers
 };
 
 struct IdxUnit {
@@ -42,18 +45,17 @@ struct IdxUnit {
 };
 
 __global__ void __launch_bounds__(IDXP_THREADS, 1)
-index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64, Hi, total_q)
-                     const __grid_constant__ CUtensorMap tmap_k,   // idx_k  (64, 128, Hi, P)
+index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64, Hi, total_q), box (64, 1, 128)
+                     const __grid_constant__ CUtensorMap tmap_k,   // idx_k  (64, 128, Hi, P), box (64, 128, 1, 1)
                      const IdxPrefillArgs a) {
   extern __shared__ __align__(1024) uint8_t dsmem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   const int head_bytes = IDXP_TILE * 64 * 2;            // 16 KiB per head tile
   const int q_bytes = a.hg * head_bytes;
-  const int k_bytes = a.hg * head_bytes;
   uint8_t* q_smem = smem;
-  uint8_t* k_smem = smem + q_bytes;
+  uint8_t* k_smem = smem + a.nqbuf * q_bytes;
 
-  __shared__ uint64_t k_full[8], k_empty[8], acc_full[4], acc_empty[4], q_full, q_empty, drain_bar;
+  __shared__ uint64_t k_full[8], k_empty[8], acc_full[2], acc_empty[2], q_full[2], q_empty[2], drain_bar;
   __shared__ uint32_t s_tmem;
   __shared__ int s_tprefix[IDXP_MAXSEQ + 1];
   __shared__ volatile int s_abort;
@@ -70,9 +72,12 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
       s_tprefix[s + 1] = acc;
     }
     for (int i = 0; i < a.stages; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
-    for (int i = 0; i < a.nbuf; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
-    mbar_init(&q_full, 1);
-    mbar_init(&q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 8);       // both epilogue warpgroups read every step
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
   }
@@ -91,12 +96,13 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
 
   // k-th unit of this CTA (snake order over the longest-first list); false when done
   auto get_unit = [&](int k, IdxUnit& u) -> bool {
-    const int r = k;  // round
     const int c = blockIdx.x;
-    const long idx = static_cast<long>(r) * G + ((r & 1) ? (G - 1 - c) : c);
+    const long idx = static_cast<long>(k) * G + ((k & 1) ? (G - 1 - c) : c);
     if (idx >= total_units) return false;
-    const int tau = total_tiles - 1 - static_cast<int>(idx / a.Hkv);  // last tiles first
-    u.g = static_cast<int>(idx % a.Hkv);
+    // group-major: all CTAs work on one group's keys at a time (they stay in L2);
+    // within a group the last (longest) query tiles come first
+    u.g = static_cast<int>(idx / total_tiles);
+    const int tau = total_tiles - 1 - static_cast<int>(idx % total_tiles);
     int lo = 0, hi = a.num_seqs - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -115,70 +121,103 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
     return true;
   };
 
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&tmap_q);
-    tma_prefetch_desc(&tmap_k);
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer warp
+    // lane 0 issues the copies; the whole warp reads the page ids of the next 32 blocks at once
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+    }
     uint32_t kit = 0, uit = 0;
-    int last_parity[8];
-    for (int i = 0; i < 8; ++i) last_parity[i] = -1;
-    int q_parity = -1;
+    uint32_t used = 0, parity_bits = 0;   // key ring slots: issued at least once / parity of the last issue
+    int q_parity0 = -1, q_parity1 = -1;
     IdxUnit u;
     for (int k = 0; get_unit(k, u) && !s_abort; ++k) {
       if (u.nblk == 0) continue;
-      if (!mbar_wait(&q_empty, (uit & 1) ^ 1, &s_abort)) break;
-      mbar_arrive_expect_tx(&q_full, q_bytes);
-      for (int hl = 0; hl < a.hg; ++hl)
-        tma_load_3d(q_smem + hl * head_bytes, &tmap_q, &q_full, 0, u.g * a.hg + hl, u.row0);
-      q_parity = uit & 1;
-      ++uit;
+      const int qb = uit % a.nqbuf;
+      const uint32_t qpar = (uit / a.nqbuf) & 1;
       bool ok = true;
-      for (int b = 0; b < u.nblk; ++b, ++kit) {
-        const int st = kit % a.stages;
-        if (!mbar_wait(&k_empty[st], ((kit / a.stages) & 1) ^ 1, &s_abort)) { ok = false; break; }
-        int page = __ldg(a.page_table + static_cast<long>(u.seq) * a.max_blocks + b);
-        if (page < 0 || page >= a.num_pages) { flag_error(MSA_DEV_BOUNDS); page = 0; }
-        mbar_arrive_expect_tx(&k_full[st], k_bytes);
-        tma_load_4d(k_smem + st * k_bytes, &tmap_k, &k_full[st], 0, 0, u.g * a.hg, page);
-        last_parity[st] = (kit / a.stages) & 1;
+      if (lane == 0) {
+        ok = mbar_wait(&q_empty[qb], qpar ^ 1, &s_abort);
+        if (ok) {
+          mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+          for (int hl = 0; hl < a.hg; ++hl)
+            tma_load_3d(q_smem + qb * q_bytes + hl * head_bytes, &tmap_q, &q_full[qb], 0, u.g * a.hg + hl, u.row0);
+          if (qb == 0) q_parity0 = static_cast<int>(qpar); else q_parity1 = static_cast<int>(qpar);
+        }
+      }
+      if (__any_sync(0xFFFFFFFFu, !ok)) break;
+      ++uit;
+      const int npair = (u.nblk + 1) >> 1;
+      int page_l = 0;
+      for (int pr = 0; pr < npair && ok; ++pr) {
+        const int b0 = 2 * pr;
+        if ((b0 & 31) == 0) {                 // page ids of blocks b0 .. b0+31
+          const int bb = b0 + lane;
+          page_l = 0;
+          if (bb < u.nblk) {
+            page_l = __ldg(a.page_table + static_cast<long>(u.seq) * a.max_blocks + bb);
+            if (page_l < 0 || page_l >= a.num_pages) { flag_error(MSA_DEV_BOUNDS); page_l = 0; }
+          }
+        }
+        const int page0 = __shfl_sync(0xFFFFFFFFu, page_l, b0 & 31);
+        int page1 = __shfl_sync(0xFFFFFFFFu, page_l, (b0 + 1) & 31);
+        if (b0 + 1 >= u.nblk) page1 = page0;  // odd block count: the second half is ignored
+        for (int hl = 0; hl < a.hg; ++hl, ++kit) {
+          const int st = kit % a.stages;
+          if (lane == 0) {
+            ok = mbar_wait(&k_empty[st], ((kit / a.stages) & 1) ^ 1, &s_abort);
+            if (ok) {
+              uint8_t* dst = k_smem + st * IDXP_STAGE_BYTES;
+              mbar_arrive_expect_tx(&k_full[st], IDXP_STAGE_BYTES);
+              tma_load_4d(dst, &tmap_k, &k_full[st], 0, 0, u.g * a.hg + hl, page0);
+              tma_load_4d(dst + head_bytes, &tmap_k, &k_full[st], 0, 0, u.g * a.hg + hl, page1);
+              used |= 1u << st;
+              parity_bits = (parity_bits & ~(1u << st)) | (((kit / a.stages) & 1u) << st);
+            }
+          }
+          if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+        }
       }
       if (!ok) break;
     }
-    if (s_abort) {  // let issued copies land before the CTA exits
+    if (lane == 0 && s_abort) {  // let issued copies land before the CTA exits
       for (int i = 0; i < a.stages; ++i)
-        if (last_parity[i] >= 0) mbar_wait_drain(&k_full[i], last_parity[i]);
-      if (q_parity >= 0) mbar_wait_drain(&q_full, q_parity);
+        if (used & (1u << i)) mbar_wait_drain(&k_full[i], (parity_bits >> i) & 1u);
+      if (q_parity0 >= 0) mbar_wait_drain(&q_full[0], q_parity0);
+      if (q_parity1 >= 0) mbar_wait_drain(&q_full[1], q_parity1);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ UMMA issuer
-    const uint32_t idesc = idesc_bf16(128, 128, false, false);
+    const uint32_t idesc = idesc_bf16(128, 256, false, false);
     const uint32_t q_addr = smem_u32(q_smem), k_addr = smem_u32(k_smem);
     uint32_t kit = 0, uit = 0, ait = 0;
     IdxUnit u;
     for (int k = 0; get_unit(k, u) && !s_abort; ++k) {
       if (u.nblk == 0) continue;
-      if (!mbar_wait(&q_full, uit & 1, &s_abort)) break;
+      const int qb = uit % a.nqbuf;
+      if (!mbar_wait(&q_full[qb], (uit / a.nqbuf) & 1, &s_abort)) break;
       ++uit;
+      const int nstep = ((u.nblk + 1) >> 1) * a.hg;
       bool ok = true;
-      for (int b = 0; b < u.nblk; ++b, ++kit, ++ait) {
+      for (int sp = 0; sp < nstep; ++sp, ++kit, ++ait) {
+        const int hl = sp % a.hg;
         const int st = kit % a.stages;
-        const int buf = ait % a.nbuf;
-        if (!mbar_wait(&acc_empty[buf], ((ait / a.nbuf) & 1) ^ 1, &s_abort)) { ok = false; break; }
+        const int buf = ait & 1;
+        if (!mbar_wait(&acc_empty[buf], ((ait >> 1) & 1) ^ 1, &s_abort)) { ok = false; break; }
         if (!mbar_wait(&k_full[st], (kit / a.stages) & 1, &s_abort)) { ok = false; break; }
         tc_fence_after();
-        for (int hl = 0; hl < a.hg; ++hl) {
-          const uint32_t d = tmem + static_cast<uint32_t>((buf * a.hg + hl) * 128);
-          const uint32_t qa = q_addr + hl * head_bytes;
-          const uint32_t ka = k_addr + st * k_bytes + hl * head_bytes;
+        const uint32_t d = tmem + static_cast<uint32_t>(buf * 256);
+        const uint32_t qa = q_addr + qb * q_bytes + hl * head_bytes;
+        const uint32_t ka = k_addr + st * IDXP_STAGE_BYTES;   // 256 key rows: two blocks
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ss(d, sdesc_sw128(qa + kk * 32, 16, 1024), sdesc_sw128(ka + kk * 32, 16, 1024), idesc,
-                         kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16_ss(d, sdesc_sw128(qa + kk * 32, 16, 1024), sdesc_sw128(ka + kk * 32, 16, 1024), idesc,
+                       kk > 0 ? 1u : 0u);
         umma_commit(&k_empty[st]);
         umma_commit(&acc_full[buf]);
       }
-      umma_commit(&q_empty);  // the query tile is free once this unit's MMAs are done
+      umma_commit(&q_empty[qb]);  // the query tile is free once this unit's MMAs are done
       if (!ok) break;
     }
     if (s_abort) {
@@ -186,52 +225,57 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
       mbar_wait_drain(&drain_bar, 0);
     }
   } else if (warp >= 2) {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue warpgroups
+    const int w = (warp - 2) >> 2;             // this warpgroup pools block 2*pair + w of every step
     const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;         // row of the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t ait = 0;
     IdxUnit u;
-    for (int k = 0; get_unit(k, u); ++k) {  // exits are warp-uniform
+    for (int k = 0; get_unit(k, u); ++k) {     // exits are warp-uniform
       if (u.nblk == 0) continue;
       const bool valid = r < u.nrows;
       const int row = u.row0 + r;
       const int p = u.ctx - u.nq + (row - u.qs);
       float* srow = a.scores + (static_cast<long>(row) * a.Hkv + u.g) * a.max_blocks;
+      const int nstep = ((u.nblk + 1) >> 1) * a.hg;
       bool ok = true;
-      for (int b = 0; b < u.nblk; ++b, ++ait) {
-        const int buf = ait % a.nbuf;
-        if (!mbar_wait_warp(&acc_full[buf], (ait / a.nbuf) & 1, &s_abort)) { ok = false; break; }
+      float tot = 0.f;
+      for (int sp = 0; sp < nstep; ++sp, ++ait) {
+        const int hl = sp % a.hg;
+        const int b = 2 * (sp / a.hg) + w;     // this warpgroup's block
+        const int buf = ait & 1;
+        if (!mbar_wait_warp(&acc_full[buf], (ait >> 1) & 1, &s_abort)) { ok = false; break; }
         tc_fence_after();
-        const int vis = p - b * a.block_size + 1;   // visible keys of block b for this row
-        float tot = 0.f;
-        for (int hl = 0; hl < a.hg; ++hl) {
-          float mx = -INFINITY;
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float v0[32], v1[32];
-            const uint32_t col = static_cast<uint32_t>((buf * a.hg + hl) * 128 + half * 64);
-            tmem_ld32(lane_addr + col, v0);
-            tmem_ld32(lane_addr + col + 32, v1);
-            tmem_ld_wait();
-            const int base = half * 64;
-            if (vis >= base + 64) {
-#pragma unroll
-              for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(v0[c], v1[c]));
-            } else {
-#pragma unroll
-              for (int c = 0; c < 32; ++c) {
-                if (base + c < vis) mx = fmaxf(mx, v0[c]);
-                if (base + 32 + c < vis) mx = fmaxf(mx, v1[c]);
-              }
-            }
-          }
-          tot += mx;
-        }
+        float v0[32], v1[32], v2[32], v3[32];  // the block's 128 scores for this row
+        const uint32_t col = lane_addr + static_cast<uint32_t>(buf * 256 + w * 128);
+        tmem_ld32(col, v0);
+        tmem_ld32(col + 32, v1);
+        tmem_ld32(col + 64, v2);
+        tmem_ld32(col + 96, v3);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        if (valid) srow[b] = tot;  // -inf when the block is past the row's current block
+        const int vis = p - b * a.block_size + 1;   // visible keys of block b for this row
+        float mx[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+        if (vis >= 128) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) mx[c & 7] = fmax3(mx[c & 7], fmaxf(v0[c], v1[c]), fmaxf(v2[c], v3[c]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            if (c < vis) mx[c & 7] = fmaxf(mx[c & 7], v0[c]);
+            if (32 + c < vis) mx[c & 7] = fmaxf(mx[c & 7], v1[c]);
+            if (64 + c < vis) mx[c & 7] = fmaxf(mx[c & 7], v2[c]);
+            if (96 + c < vis) mx[c & 7] = fmaxf(mx[c & 7], v3[c]);
+          }
+        }
+        const float hm = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], fmax3(mx[4], mx[5], mx[6]), mx[7]));
+        tot = (hl == 0) ? hm : tot + hm;
+        if (hl == a.hg - 1 && valid && b < u.nblk) __stcs(srow + b, tot);  // -inf past the row's block
       }
       if (!ok) break;
     }

@@ -137,8 +137,8 @@ msa_status_t launched() {
 
 // ---------------------------------------------------------------- workspace plans
 struct PrefillWs {
-  size_t counts, offsets, tile_offsets, cursor, total_tiles, entries, part_lse, part_o, bytes;
-  long nbuckets;
+  size_t counts, offsets, tile_offsets, cursor, total_tiles, entries, tile_rec, part_lse, part_o, bytes;
+  long nbuckets, max_tiles;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -155,6 +155,8 @@ PrefillWs prefill_plan(const msa_config_t* c, const msa_batch_t* b) {
   w.total_tiles = take(16);
   const size_t ent = static_cast<size_t>(b->total_q) * c->num_kv_heads * c->topk;
   w.entries = take(ent * 4);
+  w.max_tiles = static_cast<long>((ent + msa::ATTP_TOK - 1) / msa::ATTP_TOK) + w.nbuckets;
+  w.tile_rec = take(static_cast<size_t>(w.max_tiles) * 64);
   w.part_lse = take(static_cast<size_t>(b->total_q) * c->num_q_heads * c->topk * 4);
   w.part_o = take(static_cast<size_t>(b->total_q) * c->topk * c->num_q_heads * c->head_dim * 2);
   w.bytes = o;
@@ -263,14 +265,30 @@ msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch,
     a.hg = hg;
     a.block_size = cfg->block_size;
     a.stage_bytes = hg * 128 * 64 * 2;
-    a.stages = std::min(16, msa::IDXD_RING_BYTES / a.stage_bytes);
-    const int smem = a.stages * a.stage_bytes + 1024;
-    CUDA_TRY(set_smem(msa::index_decode_kernel, smem));
-    msa::index_decode_kernel<<<sms, msa::IDXD_THREADS, smem, stream>>>(tk, a);
-    return launched();
+    const int mq = batch->max_q_per_seq;
+    const int nqb = mq <= 1 ? 1 : mq <= 2 ? 2 : mq <= 4 ? 4 : 8;   // compile-time query bound
+    const int q_bytes = nqb * Hi * 64 * 4;
+    a.stages = std::min(16, (msa::IDXD_SMEM_BUDGET - q_bytes) / a.stage_bytes);
+    CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
+    const int smem = a.stages * a.stage_bytes + q_bytes + 1024;
+    auto go = [&](auto kernel) -> msa_status_t {
+      CUDA_TRY(set_smem(kernel, smem));
+      kernel<<<sms, msa::IDXD_THREADS, smem, stream>>>(tk, a);
+      return launched();
+    };
+    if (mq <= 1) return go(msa::index_decode_kernel<1>);
+    if (mq <= 2) return go(msa::index_decode_kernel<2>);
+    if (mq <= 4) return go(msa::index_decode_kernel<4>);
+    return go(msa::index_decode_kernel<8>);
   }
   CHECK_SUP(batch->num_seqs <= msa::IDXP_MAXSEQ, "at most %d sequences per tensor-core indexer call",
             msa::IDXP_MAXSEQ);
+  {
+    const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
+    const uint64_t strides[3] = {128, 128 * 128, static_cast<uint64_t>(Hi) * 128 * 128};
+    const uint32_t box[4] = {64, 128, 1, 1};
+    if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box)) != MSA_OK) return st;
+  }
   CUtensorMap tq;
   {
     const uint64_t dims[3] = {64, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->total_q)};
@@ -291,11 +309,11 @@ msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch,
   a.Hkv = Hkv;
   a.hg = hg;
   a.block_size = cfg->block_size;
-  const int tile_bytes = hg * 128 * 64 * 2;
-  a.stages = std::min(8, (200 * 1024 - tile_bytes) / tile_bytes);
-  a.nbuf = std::max(1, 4 / hg);
+  const int q_tile = hg * 128 * 64 * 2;
+  a.nqbuf = (2 * q_tile + 2 * msa::IDXP_STAGE_BYTES <= 200 * 1024) ? 2 : 1;
+  a.stages = std::min(8, (200 * 1024 - a.nqbuf * q_tile) / msa::IDXP_STAGE_BYTES);
   CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
-  const int smem = tile_bytes * (1 + a.stages) + 1024;
+  const int smem = a.nqbuf * q_tile + a.stages * msa::IDXP_STAGE_BYTES + 1024;
   CUDA_TRY(set_smem(msa::index_prefill_kernel, smem));
   msa::index_prefill_kernel<<<sms, msa::IDXP_THREADS, smem, stream>>>(tq, tk, a);
   return launched();
@@ -340,7 +358,7 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
             "pointers must be 16-byte aligned");
   const PrefillWs w = prefill_plan(cfg, batch);
   CHECK_ARG(workspace != nullptr && workspace_bytes >= w.bytes, "workspace too small: %zu bytes needed", w.bytes);
-  CHECK_SUP(w.nbuckets < (1L << 31), "too many (sequence, group, block) buckets");
+  CHECK_SUP(w.nbuckets < (1L << 31) && w.max_tiles < (1L << 31), "too many (sequence, group, block) buckets");
   if (batch->total_q == 0) return MSA_OK;
   char* ws = static_cast<char*>(workspace);
   const int Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, k = cfg->topk;
@@ -362,6 +380,10 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
   s.max_blocks = batch->max_blocks_per_seq;
   s.block_size = cfg->block_size;
   s.nbuckets = static_cast<int>(w.nbuckets);
+  s.tile_rec = reinterpret_cast<int4*>(ws + w.tile_rec);
+  s.page_table = batch->page_table;
+  s.num_pages = batch->num_pages;
+  s.max_tiles = static_cast<int>(w.max_tiles);
   CUDA_TRY(cudaMemsetAsync(s.counts, 0, w.nbuckets * 4, stream));
   const unsigned sgrid = static_cast<unsigned>((batch->total_q + msa::SCHED_ROWS - 1) / msa::SCHED_ROWS);
   const int ssmem = w.nbuckets <= msa::SCHED_SMEM_BUCKETS ? static_cast<int>(3 * w.nbuckets * 4) : 0;
@@ -370,6 +392,10 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
   msa::sched_scan_kernel<<<1, 1024, 0, stream>>>(s);
   if ((st = launched()) != MSA_OK) return st;
   msa::sched_count_scatter_kernel<<<sgrid, 256, ssmem, stream>>>(s, 1);
+  if ((st = launched()) != MSA_OK) return st;
+  const int sms = num_sms();
+  const long tgrid = std::min<long>((w.max_tiles + 255) / 256, 8L * sms);
+  msa::sched_tiles_kernel<<<static_cast<unsigned>(std::max<long>(1, tgrid)), 256, 0, stream>>>(s);
   if ((st = launched()) != MSA_OK) return st;
 
   CUtensorMap tq, tk, tv, tpo;
@@ -393,26 +419,15 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
     if ((st = make_map(&tpo, ws + w.part_o, 2, dims, strides, box)) != MSA_OK) return st;
   }
   msa::AttnPrefillArgs a{};
-  a.q_start = batch->q_start;
-  a.ctx_len = batch->ctx_len;
-  a.page_table = batch->page_table;
-  a.offsets = s.offsets;
-  a.tile_offsets = s.tile_offsets;
-  a.entries = s.entries;
+  a.tile_rec = s.tile_rec;
   a.total_tiles = s.total_tiles;
   a.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
-  a.num_seqs = batch->num_seqs;
-  a.total_q = batch->total_q;
   a.Hq = Hq;
-  a.Hkv = Hkv;
   a.topk = k;
-  a.max_blocks = batch->max_blocks_per_seq;
-  a.num_pages = batch->num_pages;
-  a.block_size = cfg->block_size;
-  a.nbuckets = s.nbuckets;
+  a.max_tiles = s.max_tiles;
   a.scale_log2 = softmax_scale(cfg) * 1.4426950408889634f;
   CUDA_TRY(set_smem(msa::attn_prefill_kernel, msa::ATTP_SMEM));
-  msa::attn_prefill_kernel<<<num_sms(), msa::ATTP_THREADS, msa::ATTP_SMEM, stream>>>(tq, tk, tv, tpo, a);
+  msa::attn_prefill_kernel<<<sms, msa::ATTP_THREADS, msa::ATTP_SMEM, stream>>>(tq, tk, tv, tpo, a);
   if ((st = launched()) != MSA_OK) return st;
 
   msa::MergeArgs m{};

@@ -56,19 +56,23 @@ def test_topk_matches_oracle_exactly(cuda_ok, nb, topk):
 
 # ----------------------------------------------------------------- indexer scores
 
-def _mixed_workload(seed, nq_big=True):
+def _mixed_workload(seed, nq_big=True, nq=None):
     """Several sequences, random page table, ragged tails; queries at the end
     of each context (chunked-prefill positions)."""
     ctx = [1000, 3000, 129, 5000, 256]
-    nq = [1000, 300, 129, 200, 1] if nq_big else [1, 4, 1, 3, 1]
+    if nq is None:
+        nq = [1000, 300, 129, 200, 1] if nq_big else [1, 4, 1, 3, 1]
     return gen.make_workload("mixed", seed=seed, ctx_len=ctx, nq=nq, num_q_heads=64, num_kv_heads=4,
                              idx_heads=8, topk=16, plant_frac=0.1, random_pages=True)
 
 
-@pytest.mark.parametrize("which", ["tiny", "mixed_prefill", "mixed_decode", "tiny_decode"])
+@pytest.mark.parametrize("which", ["tiny", "mixed_prefill", "mixed_decode", "tiny_decode", "decode_nq1",
+                                   "decode_nq2"])
 def test_index_scores_match_oracle(cuda_ok, which):
     if which == "tiny":
         wl = configs.tiny_prefill_2k()
+    elif which in ("decode_nq1", "decode_nq2"):
+        wl = _mixed_workload(13, nq=[1] * 5 if which == "decode_nq1" else [2, 1, 2, 2, 1])
     elif which == "tiny_decode":
         wl = gen.make_workload("tinyd", seed=5, ctx_len=[2048, 700, 4000], nq=[1, 2, 8], num_q_heads=16,
                                num_kv_heads=1, idx_heads=4, topk=4, plant_count=2, random_pages=True)

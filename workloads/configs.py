@@ -33,6 +33,11 @@ def prefill_32k(seed: int = 0) -> Workload:
                          plant_frac=0.05, **M3_HEADS)
 
 
+def prefill_8k(seed: int = 0) -> Workload:
+    """A smaller M3-shaped prefill (8192 tokens, 5% planted) for profiling."""
+    return make_workload("prefill_8k", seed=seed, ctx_len=[8192], nq=[8192], plant_frac=0.05, **M3_HEADS)
+
+
 def chunked_prefill_128k(seed: int = 0, chunk: int = None) -> List[Workload] | Workload:
     """The 8 chunks (or one of them).  Chunk c queries positions
     [16384c, 16384(c+1)) against the causal context 16384(c+1); all chunks
