@@ -27,7 +27,7 @@ EXPORTS = (
     "msa_index_scores", "msa_topk_blocks", "msa_attn_prefill", "msa_attn_decode",
     "msa_prefill_workspace_bytes", "msa_decode_workspace_bytes", "msa_get_device_status",
     "msa_set_wait_limit_ns", "msa_debug_wait_timeout", "msa_status_string", "msa_last_error",
-    "msa_version",
+    "msa_version", "msa_attn_decode_noalloc",
 )
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, MSA_ERR_DEVICE_BOUNDS = range(6)
@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "msa_topk_blocks": [cfgp, batp, P, P, P],
         "msa_attn_prefill": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
         "msa_attn_decode": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
+        "msa_attn_decode_noalloc": [cfgp, batp, P, P, P, P, P, P, P],
         "msa_prefill_workspace_bytes": [cfgp, batp],
         "msa_decode_workspace_bytes": [cfgp, batp],
         "msa_get_device_status": [P],
@@ -212,6 +213,19 @@ def attn_prefill(cfg: Config, batch: Batch, q, k_cache, v_cache, block_idx, out,
 def attn_decode(cfg: Config, batch: Batch, q, k_cache, v_cache, block_idx, out, lse=None, workspace=None,
                 stream=None) -> None:
     _attn(load_library().msa_attn_decode, cfg, batch, q, k_cache, v_cache, block_idx, out, lse, workspace, stream)
+
+
+def attn_decode_noalloc(cfg: Config, batch: Batch, q, k_cache, v_cache, block_idx, out, lse=None,
+                        stream=None) -> None:
+    """msa_attn_decode without a workspace: for callers that cannot allocate,
+    the scratch lives in a fixed 16 MiB device array inside the library (see
+    include/msa.h).  Calls that may overlap on the GPU must be serialized."""
+    lib = load_library()
+    _check(lib.msa_attn_decode_noalloc(ctypes.byref(cfg._c()), ctypes.byref(batch._c()),
+                                       _need(q, torch.bfloat16, "q"), _need(k_cache, torch.bfloat16, "k_cache"),
+                                       _need(v_cache, torch.bfloat16, "v_cache"),
+                                       _need(block_idx, torch.int32, "block_idx"), _need(out, torch.bfloat16, "out"),
+                                       _need(lse, torch.float32, "lse"), _stream(stream)))
 
 
 def device_status(stream=None) -> int:

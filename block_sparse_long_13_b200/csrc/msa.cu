@@ -509,3 +509,57 @@ msa_status_t msa_debug_wait_timeout(cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free decode attention
+// Some callers cannot hand this library a workspace: a plugin driven by a host
+// framework that passes it only input and output buffers has no allocator of
+// its own, and a serving loop may forbid cudaMalloc on the per-step path
+// (it can synchronize the device and its latency is unbounded).  For them
+// msa_attn_decode_noalloc keeps the split-K partials and counters of the
+// decode attention in this fixed device array instead.  The array is part of
+// the library's device code: every GPU that loads the library holds it until
+// the process exits.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr int kNoAllocMaxDevices = 64;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the array on the current device.  In host code the name
+// g_noalloc_scratch only stands for the symbol; the first call on each device
+// asks the runtime for the real address (cudaGetSymbolAddress) and keeps it.
+msa_status_t noalloc_scratch(void** out) {
+  int dev = -1;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MSA_ERR_UNSUPPORTED, "device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return MSA_OK;
+}
+}  // namespace
+
+extern "C" msa_status_t msa_attn_decode_noalloc(const msa_config_t* cfg, const msa_batch_t* batch, const void* q,
+                                                const void* k_cache, const void* v_cache, const int32_t* block_idx,
+                                                void* out, float* lse, cudaStream_t stream) {
+  msa_status_t st;
+  if ((st = check_config(cfg)) != MSA_OK) return st;
+  if ((st = check_batch(batch)) != MSA_OK) return st;
+  const size_t need = decode_plan(cfg, batch).bytes;
+  if (need > kNoAllocScratchBytes)
+    return fail(MSA_ERR_UNSUPPORTED,
+                "this batch needs %zu bytes of decode scratch, more than the %zu-byte static area of "
+                "msa_attn_decode_noalloc; split the batch or use msa_attn_decode with a workspace",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != MSA_OK) return st;
+  // the decode path clears its counters itself (cudaMemsetAsync, no allocation)
+  return msa_attn_decode(cfg, batch, q, k_cache, v_cache, block_idx, out, lse, scratch, kNoAllocScratchBytes,
+                         stream);
+}
+

@@ -154,6 +154,28 @@ msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, 
                              const void* k_cache, const void* v_cache, const int32_t* block_idx, void* out,
                              float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Same result as msa_attn_decode, for callers that cannot provide a workspace:
+ * a plugin that a host framework hands only its input and output buffers has
+ * no allocator to get one from, and some serving loops must not call
+ * cudaMalloc per step (it may synchronize the device and takes unbounded
+ * time).  The scratch lives in a fixed 16 MiB device array inside the library
+ * (held by every GPU that loads it until exit); this call allocates nothing.
+ * The pages describing MSA have no counterpart of this call.
+ *   - Batches whose decode scratch (msa_decode_workspace_bytes) exceeds 16 MiB
+ *     are rejected with MSA_ERR_UNSUPPORTED and a message; nothing is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) and remembers it; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; the call clears the counters it needs.  Calls that can overlap
+ *     on the GPU (different streams, or concurrent host threads) race on the
+ *     array: serialize them.
+ */
+msa_status_t msa_attn_decode_noalloc(const msa_config_t* cfg, const msa_batch_t* batch, const void* q,
+                                     const void* k_cache, const void* v_cache, const int32_t* block_idx, void* out,
+                                     float* lse, cudaStream_t stream);
+
 /* Workspace sizes (bytes) for the two attention calls; only the host fields of
  * `batch` are read.  0 means the arguments are invalid. */
 size_t msa_prefill_workspace_bytes(const msa_config_t* cfg, const msa_batch_t* batch);
