@@ -263,13 +263,19 @@ def dist_setup():
     return 0, 1, 0
 
 
-def max_over_ranks(x, ws):
+def max_over_ranks(x, ws, device="cuda"):
+    """Slowest rank's value (timings are taken per rank on its device)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_rank, ws, ms_slowest):
+    """Whole-job tokens/s: every rank processes its own replica (weak scaling)."""
+    return tokens_per_rank * ws / (ms_slowest / 1e3)
 
 
 def barrier(ws):
@@ -356,7 +362,7 @@ def main():
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, ws)
-    value = tokens * ws / (ms_max / 1e3)
+    value = job_throughput(tokens, ws, ms_max)
 
     # per-call device times (average over the timed steps) and algorithmic work
     calls = {}
@@ -451,7 +457,7 @@ def main():
         torch.cuda.synchronize()
         barrier(ws)
         ems = max_over_ranks(a0.elapsed_time(a1) / ksteps, ws)
-        e2e = {"value": tokens * ws / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+        e2e = {"value": job_throughput(tokens, ws, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": ems}
     st = msa.device_status()
 

@@ -35,8 +35,7 @@ static_assert(128 * ATTP_REGS_CTRL + 256 * ATTP_REGS_SOFTMAX <= 384 * 168, "regi
 constexpr int ATTP_TOK = 8;       // tokens per tile (x 16 heads = 128 MMA rows)
 constexpr int ATTP_G = 16;        // query heads per KV group
 constexpr int ATTP_PHASES = 4;    // tile-list phases walked in lockstep by all CTAs
-constexpr int SCHED_ROWS = 256;   // query rows per schedule CTA
-constexpr int SCHED_SMEM_BUCKETS = 4096;
+constexpr int SCHED_ROWS = 32;    // query rows per schedule CTA
 
 // ------------------------------------------------------------------ schedule
 struct SchedArgs {
@@ -58,56 +57,31 @@ __device__ __forceinline__ int entry_bucket(const SchedArgs& a, int t, int g, in
   return (s * a.Hkv + g) * a.max_blocks + b;
 }
 
-// pass = 0: count entries per bucket; pass = 1: scatter them
+// pass = 0: count entries per bucket; pass = 1: scatter them.  Buckets are
+// many (sequences x groups x blocks) and each CTA's rows hit few entries of
+// each, so the counters are global atomics; the order of entries inside a
+// bucket is arbitrary and does not change any result.
 __global__ void __launch_bounds__(256) sched_count_scatter_kernel(const SchedArgs a, int pass) {
-  extern __shared__ int sh[];  // [3][nbuckets] when nbuckets <= SCHED_SMEM_BUCKETS
-  const bool use_smem = a.nbuckets <= SCHED_SMEM_BUCKETS;
-  int* lcnt = sh;
-  int* lbase = sh + a.nbuckets;
-  int* lcur = sh + 2 * a.nbuckets;
   const int t0 = blockIdx.x * SCHED_ROWS;
   const int t1 = min(a.total_q, t0 + SCHED_ROWS);
-  if (use_smem) {
-    for (int i = threadIdx.x; i < a.nbuckets; i += blockDim.x) { lcnt[i] = 0; lcur[i] = 0; }
-    __syncthreads();
-  }
   const int per_row = a.Hkv * a.topk;
   const long e0 = static_cast<long>(t0) * per_row, e1 = static_cast<long>(t1) * per_row;
-  // entries of this CTA's rows
-  for (int round = 0; round < (use_smem && pass == 1 ? 2 : 1); ++round) {
-    for (long e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
-      const int b = __ldg(a.block_idx + e);
-      if (b < 0) continue;
-      const int t = static_cast<int>(e / per_row);
-      const int g = static_cast<int>((e / a.topk) % a.Hkv);
-      const int slot = static_cast<int>(e % a.topk);
-      const int s = find_seq(a.q_start, a.num_seqs, t);
-      const int qs = __ldg(a.q_start + s), nq = __ldg(a.q_start + s + 1) - qs;
-      const int p = __ldg(a.ctx_len + s) - nq + (t - qs);
-      if (b >= a.max_blocks || b > p / a.block_size) { flag_error(MSA_DEV_BOUNDS); continue; }
-      const int bk = entry_bucket(a, t, g, b, s);
-      if (pass == 0) {
-        if (use_smem) atomicAdd(&lcnt[bk], 1); else atomicAdd(&a.counts[bk], 1);
-      } else if (!use_smem) {
-        const int pos = atomicAdd(&a.cursor[bk], 1);
-        a.entries[pos] = (t << 6) | slot;
-      } else if (round == 0) {
-        atomicAdd(&lcnt[bk], 1);
-      } else {
-        const int pos = lbase[bk] + atomicAdd(&lcur[bk], 1);
-        a.entries[pos] = (t << 6) | slot;
-      }
-    }
-    if (use_smem) {
-      __syncthreads();
-      if (pass == 0) {
-        for (int i = threadIdx.x; i < a.nbuckets; i += blockDim.x)
-          if (lcnt[i]) atomicAdd(&a.counts[i], lcnt[i]);
-      } else if (round == 0) {
-        for (int i = threadIdx.x; i < a.nbuckets; i += blockDim.x)
-          if (lcnt[i]) lbase[i] = atomicAdd(&a.cursor[i], lcnt[i]);
-        __syncthreads();
-      }
+  for (long e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+    const int b = __ldg(a.block_idx + e);
+    if (b < 0) continue;
+    const int t = static_cast<int>(e / per_row);
+    const int g = static_cast<int>((e / a.topk) % a.Hkv);
+    const int slot = static_cast<int>(e % a.topk);
+    const int s = find_seq(a.q_start, a.num_seqs, t);
+    const int qs = __ldg(a.q_start + s), nq = __ldg(a.q_start + s + 1) - qs;
+    const int p = __ldg(a.ctx_len + s) - nq + (t - qs);
+    if (b >= a.max_blocks || b > p / a.block_size) { flag_error(MSA_DEV_BOUNDS); continue; }
+    const int bk = entry_bucket(a, t, g, b, s);
+    if (pass == 0) {
+      atomicAdd(&a.counts[bk], 1);
+    } else {
+      const int pos = atomicAdd(&a.cursor[bk], 1);
+      a.entries[pos] = (t << 6) | slot;
     }
   }
 }

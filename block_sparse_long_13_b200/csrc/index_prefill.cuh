@@ -263,7 +263,7 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
         for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
         if (vis >= 128) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) mx[c & 7] = fmax3(mx[c & 7], fmaxf(v0[c], v1[c]), fmaxf(v2[c], v3[c]));
+          for (int c = 0; c < 32; ++c) mx[c & 7] = fmax3(fmax3(mx[c & 7], v0[c], v1[c]), v2[c], v3[c]);
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {

@@ -386,12 +386,11 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
   s.max_tiles = static_cast<int>(w.max_tiles);
   CUDA_TRY(cudaMemsetAsync(s.counts, 0, w.nbuckets * 4, stream));
   const unsigned sgrid = static_cast<unsigned>((batch->total_q + msa::SCHED_ROWS - 1) / msa::SCHED_ROWS);
-  const int ssmem = w.nbuckets <= msa::SCHED_SMEM_BUCKETS ? static_cast<int>(3 * w.nbuckets * 4) : 0;
-  msa::sched_count_scatter_kernel<<<sgrid, 256, ssmem, stream>>>(s, 0);
+  msa::sched_count_scatter_kernel<<<sgrid, 256, 0, stream>>>(s, 0);
   if ((st = launched()) != MSA_OK) return st;
   msa::sched_scan_kernel<<<1, 1024, 0, stream>>>(s);
   if ((st = launched()) != MSA_OK) return st;
-  msa::sched_count_scatter_kernel<<<sgrid, 256, ssmem, stream>>>(s, 1);
+  msa::sched_count_scatter_kernel<<<sgrid, 256, 0, stream>>>(s, 1);
   if ((st = launched()) != MSA_OK) return st;
   const int sms = num_sms();
   const long tgrid = std::min<long>((w.max_tiles + 255) / 256, 8L * sms);

@@ -10,9 +10,13 @@
 //
 // "Exp-free": selection runs on the raw fp32 scores (softmax is monotone).
 // Each candidate becomes a distinct 64-bit key (order-preserving score bits,
-// then the complement of its block id), and the (topk-1)-th largest key is
-// found by an MSB-first bitwise search whose counts are warp reductions
-// (redux.sync), stopping as soon as exactly topk-1 keys lie above the probe.
+// then the complement of its block id); the answer is every key at or above
+// the (topk-1)-th largest.  One warp per row (up to 1024 blocks) first finds
+// the (topk-1)-th largest of its 32 lane maxima, a lower bound of that
+// threshold, and ranks exactly the few keys at or above it.  Wider rows, and
+// rows where that candidate set is large, run an MSB-first bitwise search
+// whose counts are warp reductions (redux.sync), stopping as soon as exactly
+// topk-1 keys lie above the probe.
 #pragma once
 #include "common.cuh"
 
@@ -33,6 +37,8 @@ topk_blocks_kernel(const float* __restrict__ scores, int32_t* __restrict__ out,
   __shared__ int s_cnt[W > 1 ? W : 1];
   __shared__ int s_sel[W > 1 ? 64 : 1];
   __shared__ int s_nsel;
+  __shared__ uint64_t s_cand[W == 1 ? 4 : 1][64];   // fast-path candidates, one area per warp
+  __shared__ uint64_t s_thr[W == 1 ? 4 : 1];
   if (row >= nrows) return;  // W == 1: whole warp leaves together; W > 1: whole CTA
   const int tid = (W == 1) ? lane : static_cast<int>(threadIdx.x);
   const int t = static_cast<int>(row / Hkv);
@@ -49,20 +55,21 @@ topk_blocks_kernel(const float* __restrict__ scores, int32_t* __restrict__ out,
   const int cur = static_cast<int>(p / block_size);
   const float* srow = scores + row * static_cast<long>(max_blocks);
 
-  // load candidates b < cur with a finite score
+  // load candidates b < cur with a finite score.  Every lane issues all NPER
+  // loads before using any (an in-bounds clamped address where b >= cur), so
+  // they are in flight together instead of one round trip each.
+  float sv[NPER];
+  const int last = cur > 0 ? cur - 1 : 0;
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) sv[i] = __ldcs(srow + min(tid + i * THREADS, last));
   uint64_t key[NPER];
   int nvalid = 0;
 #pragma unroll
   for (int i = 0; i < NPER; ++i) {
     const int b = tid + i * THREADS;
-    key[i] = 0;
-    if (b < cur) {
-      const float v = __ldg(srow + b);
-      if (v > -INFINITY) {  // excludes -inf and NaN
-        key[i] = (static_cast<uint64_t>(order_key(v)) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - b);
-        ++nvalid;
-      }
-    }
+    const bool ok = b < cur && sv[i] > -INFINITY;  // excludes -inf and NaN
+    key[i] = ok ? (static_cast<uint64_t>(order_key(sv[i])) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - b) : 0ull;
+    nvalid += ok ? 1 : 0;
   }
   auto block_sum = [&](int v) -> int {
     v = __reduce_add_sync(0xFFFFFFFFu, v);
@@ -79,7 +86,54 @@ topk_blocks_kernel(const float* __restrict__ scores, int32_t* __restrict__ out,
   const int total_valid = block_sum(nvalid);
   const bool take_all = total_valid <= m;
   uint64_t thr = 1;  // keep valid keys >= thr
-  if (!take_all && m > 0) {
+  bool found = false;
+  if (W == 1 && !take_all && m > 0 && m <= 32) {
+    // Fast path.  The m-th largest of the 32 lane maxima bounds the m-th
+    // largest key from below (those m lane maxima are m distinct keys), so the
+    // answer is among the few keys at or above it: rank those exactly.
+    uint64_t lmax = 0;
+#pragma unroll
+    for (int i = 0; i < NPER; ++i) lmax = key[i] > lmax ? key[i] : lmax;
+    uint64_t lo = 0;
+    for (int bit = 63; bit >= 0; --bit) {
+      const uint64_t probe = lo | (1ull << bit);
+      const int c = __popc(__ballot_sync(0xFFFFFFFFu, lmax >= probe));
+      if (c >= m) {
+        lo = probe;
+        if (c == m) break;
+      }
+    }
+    if (lo != 0) {
+      int cl = 0;
+#pragma unroll
+      for (int i = 0; i < NPER; ++i) cl += (key[i] >= lo) ? 1 : 0;
+      int incl = cl;  // inclusive prefix over lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      const int ncand = __shfl_sync(0xFFFFFFFFu, incl, 31);
+      if (ncand <= 64) {
+        uint64_t* cand = s_cand[warp];
+        int at = incl - cl;
+#pragma unroll
+        for (int i = 0; i < NPER; ++i)
+          if (key[i] >= lo) cand[at++] = key[i];
+        __syncwarp();
+        for (int c = lane; c < ncand; c += 32) {
+          const uint64_t kc = cand[c];
+          int above = 0;
+          for (int d = 0; d < ncand; ++d) above += (cand[d] > kc) ? 1 : 0;
+          if (above == m - 1) s_thr[warp] = kc;   // exactly one candidate: keys are distinct
+        }
+        __syncwarp();
+        thr = s_thr[warp];
+        found = true;
+      }
+    }
+  }
+  if (!take_all && m > 0 && !found) {
     uint64_t prefix = 0;
     for (int bit = 63; bit >= 0; --bit) {
       const uint64_t probe = prefix | (1ull << bit);
