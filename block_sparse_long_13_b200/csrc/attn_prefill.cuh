@@ -17,8 +17,10 @@
 // tiles of the same bucket.  S = Q K^T and O = P V run on tcgen05 with fp32
 // accumulators in TMEM; a 4-warp softmax group reads S rows from TMEM (thread
 // = row), masks keys after the query position (only the query's own block
-// has any), writes P as bf16 into a swizzled shared tile, and later stores
-// O / l (bf16) and lse = m + ln l as the partial of (t, head, slot).
+// has any), writes P as bf16 back into TMEM, from where the P V MMA reads
+// it (operand A in TMEM: shared-memory bandwidth is left to the S = Q K^T
+// operands and the V tile), and later stores O / l (bf16) and lse = m + ln l
+// as the partial of (t, head, slot).
 //
 // Phase 2 (merge): out(t, h) = sum_slots exp(lse_s - L) O_s with
 // L = log sum_s exp(lse_s); lse(t, h) = L.
@@ -186,11 +188,12 @@ __device__ __forceinline__ void load_rec(const int4* base, int tile, TileRec& r)
   r.ent[4] = d.x; r.ent[5] = d.y; r.ent[6] = d.z; r.ent[7] = d.w;
 }
 
-// shared memory plan (bytes, 1024-aligned): Q[3] 96K | K 32K | V 32K | P[2] 64K
-// P[w] also stages warpgroup w's O tile for the TMA store once PV has read P.
+// shared memory plan (bytes, 1024-aligned): Q[3] 96K | K 32K | V 32K | O staging[2] 64K
 constexpr int ATTP_QBUF = 3;      // gathered query tiles in flight (the gather latency needs > 2)
-constexpr int ATTP_QBYTES = 32768, ATTP_KVBYTES = 32768;
-constexpr int ATTP_SMEM = ATTP_QBUF * ATTP_QBYTES + 2 * ATTP_KVBYTES + 2 * 32768 + 1024;
+constexpr int ATTP_QBYTES = 32768, ATTP_KVBYTES = 32768, ATTP_STAGE = 32768;
+constexpr int ATTP_SMEM = ATTP_QBUF * ATTP_QBYTES + 2 * ATTP_KVBYTES + 2 * ATTP_STAGE + 1024;
+// TMEM columns: S[2] (fp32) at 0 / 128, P[2] (bf16 pairs) at 256 / 320, O (fp32) at 384
+constexpr uint32_t ATTP_TM_S = 0, ATTP_TM_P = 256, ATTP_TM_O = 384;
 
 __global__ void __launch_bounds__(ATTP_THREADS, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [total_q*Hq][128]
@@ -203,13 +206,15 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
   uint8_t* q_s = smem;                                  // 3 x 32 KiB: [half][128 rows][64]
   uint8_t* k_s = q_s + ATTP_QBUF * ATTP_QBYTES;         // [half][128 keys][64]
   uint8_t* v_s = k_s + ATTP_KVBYTES;                    // [half][128 keys][64]
-  uint8_t* p_s = v_s + ATTP_KVBYTES;                    // 2 x 32 KiB: [half][128 rows][64 keys]
+  uint8_t* o_s = v_s + ATTP_KVBYTES;                    // 2 x 32 KiB: [half][128 rows][64 dims]
 
-  __shared__ uint64_t kv_full, kv_empty, q_full[ATTP_QBUF], q_empty[ATTP_QBUF], s_full[2], s_empty[2], p_full[2],
-      p_empty[2], o_full[2], o_empty[2], drain_bar;
+  // Per warpgroup w (its own tile sequence, so a parity never runs two phases ahead): s_full[w] S is in
+  // TMEM, p_full[w] P is in TMEM (one arrival per warp), o_full[w] the O accumulator holds its tile.
+  // o_empty: O has been read (one arrival per warp); only the UMMA thread waits on it, in tile order.
+  __shared__ uint64_t kv_full, kv_empty, q_full[ATTP_QBUF], q_empty[ATTP_QBUF], s_full[2], p_full[2], o_full[2],
+      o_empty, drain_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
-  __shared__ int s_ent[2][2][ATTP_TOK];   // per warpgroup, two tiles: (t << 6 | slot) of each entry
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -222,17 +227,15 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
       mbar_init(&p_full[i], 4);
-      mbar_init(&p_empty[i], 1);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], 4);
     }
+    mbar_init(&o_empty, 4);
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&s_tmem, 512);  // S[2] at columns 0/128, O[2] at 256/384
+    tmem_alloc(&s_tmem, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -333,23 +336,24 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ UMMA issuer
+    // Tile i: S(i) = Q K^T into S[i % 2] (A and B from shared memory), then O = P(i-1) V with
+    // P(i-1) read from TMEM.  tcgen05.commit tracks every earlier MMA of this thread, so the
+    // s_full(i) signal also means PV(i-2) has finished reading P[i % 2].
     const uint32_t id_s = idesc_bf16(128, 128, false, false);
     const uint32_t id_pv = idesc_bf16(128, 128, false, true);
-    const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s), pa = smem_u32(p_s);
+    const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s);
     int cur_bucket = -1;
     uint32_t kvit = 0;
     bool pv_pending = false;
-    auto issue_pv = [&](int j) -> bool {  // O[j%2] = P[j%2] V
+    auto issue_pv = [&](int j) -> bool {  // O = P[j%2] V
       const int pb = j & 1;
       if (!mbar_wait(&p_full[pb], (j >> 1) & 1, &s_abort)) return false;
-      if (!mbar_wait(&o_empty[pb], ((j >> 1) & 1) ^ 1, &s_abort)) return false;
+      if (!mbar_wait(&o_empty, (j & 1) ^ 1, &s_abort)) return false;   // tile j-1's O has been read
       tc_fence_after();
-      const uint32_t d = tmem + 256 + pb * 128;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t adesc = sdesc_sw128(pa + pb * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
         const uint64_t bdesc = sdesc_sw128(va + kk * 2048, 16384, 1024);
-        umma_bf16_ss(d, adesc, bdesc, id_pv, kk > 0 ? 1u : 0u);
+        umma_bf16_ts(tmem + ATTP_TM_O, tmem + ATTP_TM_P + pb * 64 + kk * 8, bdesc, id_pv, kk > 0 ? 1u : 0u);
       }
       umma_commit(&o_full[pb]);
       return true;
@@ -371,9 +375,8 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
       }
       const int qb = i % ATTP_QBUF, sb = i & 1;
       if (!mbar_wait(&q_full[qb], (i / ATTP_QBUF) & 1, &s_abort)) break;
-      if (!mbar_wait(&s_empty[sb], ((i >> 1) & 1) ^ 1, &s_abort)) break;
       tc_fence_after();
-      const uint32_t d = tmem + sb * 128;
+      const uint32_t d = tmem + ATTP_TM_S + sb * 128;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -394,18 +397,18 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
   } else {
     regs_inc<ATTP_REGS_SOFTMAX>();
     // ------------------------------------------------------------ two softmax + epilogue warpgroups
-    // warpgroup w takes the CTA's tiles i = w, w + 2, ...; it owns Q/S/P/O buffers w
+    // Warpgroup w takes the CTA's tiles i = w, w + 2, ...; it owns S[w], P[w] and staging buffer w.
+    // Every warp runs on its own (its 32 TMEM lanes = 2 entries x 16 heads): it waits, arrives and
+    // stores its rows without waiting for the other warps.
     const int w = (warp - 4) >> 2;
-    const int bar = 1 + w;                        // named barrier of this warpgroup
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;            // MMA row = entry * 16 + head
     const int e = r >> 4, h = r & 15;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const bool issuer = (warp == 4 + 4 * w && lane == 0);
     const float LN2 = 0.69314718055994531f;
     const float sc = a.scale_log2;
     const uint64_t pol_stream = l2_policy_evict_first();
-    uint8_t* pbuf = p_s + w * 32768;
+    uint8_t* stage = o_s + w * ATTP_STAGE;
     const int nj = (ntile - w + 1) / 2;
     // the fields this row needs of its tiles, prefetched one tile ahead
     struct RowRec { int g, b, off, n, ent; };
@@ -420,7 +423,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
     };
     RowRec nxt{};
     if (nj > 0) nxt = load_row(tile_of(w));
-    for (int j = 0; j < nj; ++j) {               // every exit decision is uniform over the warpgroup
+    for (int j = 0; j < nj; ++j) {               // exit decisions are uniform over the warp
       const int i = 2 * j + w;
       const RowRec rec = nxt;
       if (j + 1 < nj) nxt = load_row(tile_of(i + 2));
@@ -428,22 +431,17 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
       const int ent = rec.ent;
       const int t = ent >> 6, slot = ent & 63;
       const int vis = valid ? min(128, t + rec.off - rec.b * 128 + 1) : 128;  // visible keys of the block
-      if (valid && h == 0) s_ent[w][j & 1][e] = ent;
-      const uint32_t par = static_cast<uint32_t>(j & 1);
 
       // ---- S = Q K^T is in TMEM: the row's 128 scores in registers, max over the visible keys
-      if (!mbar_wait_group(&s_full[w], par, &s_abort, bar, 128)) break;
+      if (!mbar_wait_warp(&s_full[w], static_cast<uint32_t>(j & 1), &s_abort)) break;
       tc_fence_after();
-      const uint32_t s_addr = lane_addr + w * 128;
+      const uint32_t s_addr = lane_addr + ATTP_TM_S + w * 128;
       float v0[32], v1[32], v2[32], v3[32];
       tmem_ld32(s_addr, v0);
       tmem_ld32(s_addr + 32, v1);
       tmem_ld32(s_addr + 64, v2);
       tmem_ld32(s_addr + 96, v3);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[w]);    // S[w] has been read
       if (vis < 128) {                            // the query's own block: keys after it do not count
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -460,71 +458,74 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
       for (int c = 0; c < 32; ++c) mx[c & 7] = fmax3(mx[c & 7], fmaxf(v0[c], v1[c]), fmaxf(v2[c], v3[c]));
       const float m = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], fmax3(mx[4], mx[5], mx[6]), mx[7]));
       const float mc = (m > -INFINITY) ? m * sc : 0.f;   // -inf only on rows past the tile's entries
-      // ---- P = exp2(scale * S - max) as bf16 into P[w] (free once the last stores from it were read)
-      if (issuer) bulk_wait_read_all();
-      named_bar_sync(bar, 128);
+      // ---- P = exp2(scale * S - max) as bf16 pairs into P[w] (TMEM), two halves of 64 keys
       float l0 = 0.f, l1 = 0.f;
 #pragma unroll
-      for (int q8 = 0; q8 < 16; ++q8) {
-        float pe[8];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int c = q8 * 8 + u;
-          const float x = c < 32 ? v0[c] : c < 64 ? v1[c - 32] : c < 96 ? v2[c - 64] : v3[c - 96];
-          pe[u] = exp2f(fmaf(x, sc, -mc));        // exp2(-inf) = 0 for masked keys
+        for (int q2 = 0; q2 < 32; ++q2) {
+          const int c = half * 64 + q2 * 2;
+          const float x0 = c < 32 ? v0[c] : c < 64 ? v1[c - 32] : c < 96 ? v2[c - 64] : v3[c - 96];
+          const float x1 = c + 1 < 32 ? v0[c + 1] : c + 1 < 64 ? v1[c - 31] : c + 1 < 96 ? v2[c - 63] : v3[c - 95];
+          const float p0 = exp2f(fmaf(x0, sc, -mc)), p1 = exp2f(fmaf(x1, sc, -mc));   // exp2(-inf) = 0
+          if (q2 & 1) l1 += p0 + p1; else l0 += p0 + p1;
+          pk[q2] = pack_bf16(p0, p1);
         }
-        l0 += (pe[0] + pe[1]) + (pe[2] + pe[3]);
-        l1 += (pe[4] + pe[5]) + (pe[6] + pe[7]);
-        uint4 wv;
-        wv.x = pack_bf16(pe[0], pe[1]);
-        wv.y = pack_bf16(pe[2], pe[3]);
-        wv.z = pack_bf16(pe[4], pe[5]);
-        wv.w = pack_bf16(pe[6], pe[7]);
-        *reinterpret_cast<uint4*>(pbuf + (q8 >> 3) * 16384 + sw128_offset(r, (q8 & 7) * 16)) = wv;
+        tmem_st32(lane_addr + ATTP_TM_P + w * 64 + half * 32, pk);
       }
-      const float l = l0 + l1;
-      fence_proxy_async_smem();                   // P visible to the tensor core
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[w]);
-
-      // ---- O = P V is in TMEM: O / l as bf16, staged in P[w] for the TMA store
-      if (!mbar_wait_group(&o_full[w], par, &s_abort, bar, 128)) break;
-      tc_fence_after();
-      const float inv = 1.f / l;
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
-        tmem_ld32(lane_addr + 256 + w * 128 + c4 * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const int col = c4 * 32 + q8 * 8;       // output dims col .. col+7
-          uint4 wv;
-          wv.x = pack_bf16(v[q8 * 8 + 0] * inv, v[q8 * 8 + 1] * inv);
-          wv.y = pack_bf16(v[q8 * 8 + 2] * inv, v[q8 * 8 + 3] * inv);
-          wv.z = pack_bf16(v[q8 * 8 + 4] * inv, v[q8 * 8 + 5] * inv);
-          wv.w = pack_bf16(v[q8 * 8 + 6] * inv, v[q8 * 8 + 7] * inv);
-          *reinterpret_cast<uint4*>(pbuf + (col >> 6) * 16384 + sw128_offset(r, (col & 63) * 2)) = wv;
-        }
-      }
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[w]);
+      if (lane == 0) mbar_arrive(&p_full[w]);
+      const float l = l0 + l1;
+
+      // ---- O = P V is in TMEM: read it, release the accumulator, then O / l as bf16 to this warp's rows
+      if (!mbar_wait_warp(&o_full[w], static_cast<uint32_t>(j & 1), &s_abort)) break;
+      tc_fence_after();
+      float o0[32], o1[32], o2[32], o3[32];
+      tmem_ld32(lane_addr + ATTP_TM_O, o0);
+      tmem_ld32(lane_addr + ATTP_TM_O + 32, o1);
+      tmem_ld32(lane_addr + ATTP_TM_O + 64, o2);
+      tmem_ld32(lane_addr + ATTP_TM_O + 96, o3);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty);
+      if (lane == 0) bulk_wait_read_all();        // this warp's previous stores have left its staging rows
+      __syncwarp();
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int q8 = 0; q8 < 16; ++q8) {
+        const int col = q8 * 8;                   // output dims col .. col+7
+        const float* ov = q8 < 4 ? o0 + col : q8 < 8 ? o1 + col - 32 : q8 < 12 ? o2 + col - 64 : o3 + col - 96;
+        uint4 wv;
+        wv.x = pack_bf16(ov[0] * inv, ov[1] * inv);
+        wv.y = pack_bf16(ov[2] * inv, ov[3] * inv);
+        wv.z = pack_bf16(ov[4] * inv, ov[5] * inv);
+        wv.w = pack_bf16(ov[6] * inv, ov[7] * inv);
+        *reinterpret_cast<uint4*>(stage + (col >> 6) * 16384 + sw128_offset(r, (col & 63) * 2)) = wv;
+      }
       if (valid)
         a.part_lse[(static_cast<long>(t) * a.Hq + rec.g * ATTP_G + h) * a.topk + slot] = (mc + log2f(l)) * LN2;
       fence_proxy_async_smem();
-      named_bar_sync(bar, 128);
-      if (issuer) {
-        for (int ee = 0; ee < rec.n; ++ee) {
-          const int en = s_ent[w][j & 1][ee];
-          const int y = ((en >> 6) * a.topk + (en & 63)) * a.Hq + rec.g * ATTP_G;
-          tma_store_2d_hint(&tmap_po, pbuf + ee * 2048, 0, y, pol_stream);
-          tma_store_2d_hint(&tmap_po, pbuf + 16384 + ee * 2048, 64, y, pol_stream);
+      const int ent_hi = __shfl_sync(0xFFFFFFFFu, ent, 16);   // entry 2*quarter + 1 (lanes 16..31)
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int ee = 2 * quarter + k2;
+          if (ee < rec.n) {
+            const int en = k2 ? ent_hi : ent;
+            const int y = ((en >> 6) * a.topk + (en & 63)) * a.Hq + rec.g * ATTP_G;
+            tma_store_2d_hint(&tmap_po, stage + ee * 2048, 0, y, pol_stream);
+            tma_store_2d_hint(&tmap_po, stage + 16384 + ee * 2048, 64, y, pol_stream);
+          }
         }
         bulk_commit();
       }
     }
-    if (issuer) bulk_wait_all();                  // partial stores complete before exit
+    if (lane == 0) bulk_wait_all();               // partial stores complete before exit
   }
   __syncwarp();
   tc_fence_before();
