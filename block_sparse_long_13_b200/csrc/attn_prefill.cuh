@@ -174,20 +174,6 @@ struct AttnPrefillArgs {
   float scale_log2;
 };
 
-struct TileRec {
-  int bucket, kv_y, g, b, off, n;
-  int ent[ATTP_TOK];
-};
-
-__device__ __forceinline__ void load_rec(const int4* base, int tile, TileRec& r) {
-  const int4* p = base + static_cast<long>(tile) * 4;
-  const int4 a = __ldg(p), b = __ldg(p + 1), c = __ldg(p + 2), d = __ldg(p + 3);
-  r.bucket = a.x; r.kv_y = a.y; r.g = a.z; r.b = a.w;
-  r.off = b.x; r.n = b.y;
-  r.ent[0] = c.x; r.ent[1] = c.y; r.ent[2] = c.z; r.ent[3] = c.w;
-  r.ent[4] = d.x; r.ent[5] = d.y; r.ent[6] = d.z; r.ent[7] = d.w;
-}
-
 // shared memory plan (bytes, 1024-aligned): Q[3] 96K | K 32K | V 32K | O staging[2] 64K
 constexpr int ATTP_QBUF = 3;      // gathered query tiles in flight (the gather latency needs > 2)
 constexpr int ATTP_QBYTES = 32768, ATTP_KVBYTES = 32768, ATTP_STAGE = 32768;
@@ -272,64 +258,89 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
 
   if (warp < 4) {
   regs_dec<ATTP_REGS_CTRL>();
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&tmap_q);
-    tma_prefetch_desc(&tmap_k);
-    tma_prefetch_desc(&tmap_v);
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer warp
+    // Tile records arrive 32 at a time (one per lane, a single coalesced load), so no record
+    // fetch sits on the issue path; lanes 0..15 issue the tile's query-row copies in parallel.
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+    }
     int cur_bucket = -1;
     uint32_t kvit = 0;
     int kv_parity = -1;
-    uint32_t q_used = 0, q_parity_bits = 0;   // per query buffer: issued at least once / parity of the last issue
-    TileRec nxt;
-    if (ntile > 0) load_rec(a.tile_rec, tile_of(0), nxt);
-    for (int i = 0; i < ntile && !s_abort; ++i) {
-      const TileRec r = nxt;
-      if (i + 1 < ntile) load_rec(a.tile_rec, tile_of(i + 1), nxt);  // in flight while this tile is issued
-      if (r.bucket != cur_bucket) {
-        if (!mbar_wait(&kv_empty, (kvit & 1) ^ 1, &s_abort)) break;
-        mbar_arrive_expect_tx(&kv_full, 2 * ATTP_KVBYTES);
-        tma_load_2d(k_s, &tmap_k, &kv_full, 0, r.kv_y);
-        tma_load_2d(k_s + 16384, &tmap_k, &kv_full, 64, r.kv_y);
-        tma_load_2d(v_s, &tmap_v, &kv_full, 0, r.kv_y);
-        tma_load_2d(v_s + 16384, &tmap_v, &kv_full, 64, r.kv_y);
-        kv_parity = kvit & 1;
+    uint32_t q_used = 0, q_parity_bits = 0;   // lane 0: per query buffer, issued at least once / parity of the last issue
+    // A group's query rows are gathered again by every block they selected: keep them in L2; a K/V
+    // block is read by the one or two CTAs that walk its bucket: let it go first.
+    const uint64_t pol_q = l2_policy_evict_last(), pol_kv = l2_policy_evict_first();
+    int4 ra = make_int4(-1, 0, 0, 0), rb = make_int4(0, 0, 0, 0), rc = rb, rd = rb;   // record of tile (batch + lane)
+    for (int i = 0; i < ntile; ++i) {
+      if (__any_sync(0xFFFFFFFFu, s_abort != 0)) break;
+      if ((i & 31) == 0 && i + lane < ntile) {
+        const int4* p = a.tile_rec + static_cast<long>(tile_of(i + lane)) * 4;
+        ra = __ldg(p); rb = __ldg(p + 1); rc = __ldg(p + 2); rd = __ldg(p + 3);
+      }
+      const int src = i & 31;
+      const int bucket = __shfl_sync(0xFFFFFFFFu, ra.x, src);
+      const int kv_y = __shfl_sync(0xFFFFFFFFu, ra.y, src);
+      const int g = __shfl_sync(0xFFFFFFFFu, ra.z, src);
+      const int n = __shfl_sync(0xFFFFFFFFu, rb.y, src);
+      // the tile's entries (t << 6 | slot)
+      const int e0 = __shfl_sync(0xFFFFFFFFu, rc.x, src), e1 = __shfl_sync(0xFFFFFFFFu, rc.y, src);
+      const int e2 = __shfl_sync(0xFFFFFFFFu, rc.z, src), e3 = __shfl_sync(0xFFFFFFFFu, rc.w, src);
+      const int e4 = __shfl_sync(0xFFFFFFFFu, rd.x, src), e5 = __shfl_sync(0xFFFFFFFFu, rd.y, src);
+      const int e6 = __shfl_sync(0xFFFFFFFFu, rd.z, src), e7 = __shfl_sync(0xFFFFFFFFu, rd.w, src);
+      // next tile's bucket (when its record is in this batch) for the K/V L2 prefetch
+      const int nb_bucket = __shfl_sync(0xFFFFFFFFu, ra.x, (src + 1) & 31);
+      const int nb_kv_y = __shfl_sync(0xFFFFFFFFu, ra.y, (src + 1) & 31);
+      bool ok = true;
+      if (bucket != cur_bucket) {
+        if (lane == 0) {
+          ok = mbar_wait(&kv_empty, (kvit & 1) ^ 1, &s_abort);
+          if (ok) {
+            mbar_arrive_expect_tx(&kv_full, 2 * ATTP_KVBYTES);
+            tma_load_2d_hint(k_s, &tmap_k, &kv_full, 0, kv_y, pol_kv);
+            tma_load_2d_hint(k_s + 16384, &tmap_k, &kv_full, 64, kv_y, pol_kv);
+            tma_load_2d_hint(v_s, &tmap_v, &kv_full, 0, kv_y, pol_kv);
+            tma_load_2d_hint(v_s + 16384, &tmap_v, &kv_full, 64, kv_y, pol_kv);
+            kv_parity = kvit & 1;
+          }
+        }
         ++kvit;
-        cur_bucket = r.bucket;
+        cur_bucket = bucket;
+        if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
       }
       const int qb = i % ATTP_QBUF;
       const uint32_t qpar = static_cast<uint32_t>((i / ATTP_QBUF) & 1);
-      if (!mbar_wait(&q_empty[qb], qpar ^ 1u, &s_abort)) break;
-      mbar_arrive_expect_tx(&q_full[qb], r.n * 4096);
-#pragma unroll
-      for (int e = 0; e < ATTP_TOK; ++e) {
-        if (e < r.n) {
-          const int y = (r.ent[e] >> 6) * a.Hq + r.g * ATTP_G;
-          tma_load_2d(q_s + qb * ATTP_QBYTES + e * 2048, &tmap_q, &q_full[qb], 0, y);
-          tma_load_2d(q_s + qb * ATTP_QBYTES + 16384 + e * 2048, &tmap_q, &q_full[qb], 64, y);
+      if (lane == 0) {
+        ok = mbar_wait(&q_empty[qb], qpar ^ 1u, &s_abort);
+        if (ok) {
+          mbar_arrive_expect_tx(&q_full[qb], n * 4096);
+          q_used |= 1u << qb;
+          q_parity_bits = (q_parity_bits & ~(1u << qb)) | (qpar << qb);
         }
       }
-      q_used |= 1u << qb;
-      q_parity_bits = (q_parity_bits & ~(1u << qb)) | (qpar << qb);
-      // warm L2 with the next tile's query rows (and its K/V when the bucket changes)
-      if (i + 1 < ntile) {
-#pragma unroll
-        for (int e = 0; e < ATTP_TOK; ++e) {
-          if (e < nxt.n) {
-            const int y = (nxt.ent[e] >> 6) * a.Hq + nxt.g * ATTP_G;
-            tma_prefetch_l2_2d(&tmap_q, 0, y);
-            tma_prefetch_l2_2d(&tmap_q, 64, y);
-          }
-        }
-        if (nxt.bucket != r.bucket) {
-          tma_prefetch_l2_2d(&tmap_k, 0, nxt.kv_y);
-          tma_prefetch_l2_2d(&tmap_k, 64, nxt.kv_y);
-          tma_prefetch_l2_2d(&tmap_v, 0, nxt.kv_y);
-          tma_prefetch_l2_2d(&tmap_v, 64, nxt.kv_y);
-        }
+      if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
+      // query rows of the tile's entries (MMA row 16e + head), [half][128 rows][64 dims] swizzled:
+      // lane 2e + half issues entry e's half
+      {
+        const int el = lane >> 1, half = lane & 1;
+        const int en = el == 0 ? e0 : el == 1 ? e1 : el == 2 ? e2 : el == 3 ? e3 : el == 4 ? e4 : el == 5 ? e5
+                     : el == 6 ? e6 : e7;
+        if (lane < 2 * ATTP_TOK && el < n)
+          tma_load_2d_hint(q_s + qb * ATTP_QBYTES + half * 16384 + el * 2048, &tmap_q, &q_full[qb], half * 64,
+                           (en >> 6) * a.Hq + g * ATTP_G, pol_q);
+      }
+      // warm L2 with the next bucket's K/V
+      if (lane == 0 && i + 1 < ntile && src != 31 && nb_bucket != bucket) {
+        tma_prefetch_l2_2d(&tmap_k, 0, nb_kv_y);
+        tma_prefetch_l2_2d(&tmap_k, 64, nb_kv_y);
+        tma_prefetch_l2_2d(&tmap_v, 0, nb_kv_y);
+        tma_prefetch_l2_2d(&tmap_v, 64, nb_kv_y);
       }
     }
-    if (s_abort) {
+    if (lane == 0 && s_abort) {                  // let issued copies land before the CTA exits
       if (kv_parity >= 0) mbar_wait_drain(&kv_full, kv_parity);
       for (int j = 0; j < ATTP_QBUF; ++j)
         if (q_used & (1u << j)) mbar_wait_drain(&q_full[j], (q_parity_bits >> j) & 1u);
