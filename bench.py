@@ -56,7 +56,7 @@ def peaks():
 class Part:
     """One batch through the three calls (indexer, top-k, attention)."""
 
-    def __init__(self, name, wl, caches, kind, out_rows=None):
+    def __init__(self, name, wl, caches, kind, out_rows=None, fused=False):
         import block_sparse_long_13_b200 as msa
         self.msa = msa
         self.name, self.wl, self.kind = name, wl, kind
@@ -69,24 +69,31 @@ class Part:
         self.q = gen.query_rows(wl, gen.TID_Q, device=dev)
         self.idx_q = gen.query_rows(wl, gen.TID_IDX_Q, device=dev)
         T, G, nb = wl.total_q, wl.num_kv_heads, wl.max_blocks
-        self.scores = torch.empty((T, G, nb), dtype=torch.float32, device=dev)
         self.sel = torch.empty((T, G, wl.topk), dtype=torch.int32, device=dev)
         self.out = torch.empty_like(self.q) if out_rows is None else out_rows
         self.lse = torch.empty((T, wl.num_q_heads), dtype=torch.float32, device=dev)
         wsb = (msa.prefill_workspace_bytes if kind == "prefill" else msa.decode_workspace_bytes)(self.cfg, self.batch)
         self.ws_bytes = wsb
         self.ws = None
-        self.launches = 7 if kind == "prefill" else 3
+        # prefill: indexer and top-k in one call (msa_index_topk) when asked
+        self.fused = fused and kind == "prefill" and wl.topk <= 16
+        self.scores = None if self.fused else torch.empty((T, G, nb), dtype=torch.float32, device=dev)
+        # kernels of ours per run: indexer (+ top-k), then attention: prefill = schedule (4 kernels),
+        # block-major attention, merge; decode = one kernel
+        self.launches = (1 if self.fused else 2) + (6 if kind == "prefill" else 1)
         self.pos = wl.positions()
 
     def run(self, ws, ev=None, stream=None, stop_after="attn"):
         m = self.msa
         if ev is not None:
             ev[0].record(stream)
-        m.index_scores(self.cfg, self.batch, self.idx_q, self.caches["idx_k"], self.scores)
+        if self.fused:
+            m.index_topk(self.cfg, self.batch, self.idx_q, self.caches["idx_k"], self.sel)
+        else:
+            m.index_scores(self.cfg, self.batch, self.idx_q, self.caches["idx_k"], self.scores)
         if ev is not None:
             ev[1].record(stream)
-        if stop_after != "index":
+        if stop_after != "index" and not self.fused:
             m.topk_blocks(self.cfg, self.batch, self.scores, self.sel)
         if ev is not None:
             ev[2].record(stream)
@@ -123,9 +130,10 @@ class Part:
         return {"bytes": float(cur.sum()) * self.wl.num_kv_heads * 4 + self.sel.numel() * 4}
 
 
-def build_parts(name, batch=None):
+def build_parts(name, batch=None, fused=False):
     """Device inputs of a workload: list of Part (in order).  `batch` shrinks
-    a decode workload (fewer sequences, same shapes) for profiling runs."""
+    a decode workload (fewer sequences, same shapes) for profiling runs;
+    `fused` selects msa_index_topk for prefill (else the two calls)."""
     parts = []
     if name in ("msa_128k_1m", "chunked_prefill_128k", "prefill_128k_last_chunk"):
         chunks = configs.chunked_prefill_128k()
@@ -137,7 +145,7 @@ def build_parts(name, batch=None):
         out_all = torch.empty((len(which) * 16384, 64, 128), dtype=torch.bfloat16, device="cuda")
         for n, c in enumerate(which):
             parts.append(Part(f"prefill128k/c{c}", chunks[c], caches, "prefill",
-                              out_all[n * 16384:(n + 1) * 16384]))
+                              out_all[n * 16384:(n + 1) * 16384], fused=fused))
     if name in ("msa_128k_1m", "decode_128k", "decode_1m", "verify_ragged"):
         for dn in (("decode_128k", "decode_1m") if name == "msa_128k_1m" else (name,)):
             wl = configs.ALL[dn](batch=batch) if batch else configs.ALL[dn]()
@@ -150,7 +158,7 @@ def build_parts(name, batch=None):
         caches = {"k": gen.paged_cache(wl, gen.TID_K, device="cuda"),
                   "v": gen.paged_cache(wl, gen.TID_V, device="cuda"),
                   "idx_k": gen.paged_cache(wl, gen.TID_IDX_K, device="cuda")}
-        parts.append(Part(name, wl, caches, "prefill"))
+        parts.append(Part(name, wl, caches, "prefill", fused=fused))
     return parts
 
 
@@ -314,6 +322,8 @@ def main():
                     help="profiling: run the step only up to this call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fused-prefill", action="store_true",
+                    help="prefill indexer and top-k in one call (msa_index_topk) instead of the two calls")
     args = ap.parse_args()
     rank, ws, local = dist_setup()
     if args.impl == "reference":
@@ -327,7 +337,7 @@ def main():
     import block_sparse_long_13_b200 as msa
     msa.load_library()  # fails loudly when the CUDA library is missing
 
-    parts = build_parts(args.workload, args.batch)
+    parts = build_parts(args.workload, args.batch, fused=args.fused_prefill)
     stream = torch.cuda.current_stream()
     ws_bytes = max(p.ws_bytes for p in parts) if args.stop_after == "attn" else 0
     workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
@@ -372,20 +382,22 @@ def main():
         t_att = statistics.mean(evs[k][i][2].elapsed_time(evs[k][i][3]) for k in range(args.steps))
         calls[p.name] = {"index_ms": t_idx, "topk_ms": t_top, "attn_ms": t_att,
                          "index": p.index_work(), "attn": p.attn_work(), "topk": p.topk_work(), "kind": p.kind,
-                         "tokens": p.wl.total_q}
+                         "tokens": p.wl.total_q, "fused": p.fused}
     pk = peaks()
     # dominant call type over the step
     agg = {}
     for name, c in calls.items():
         for key in ("index", "topk", "attn"):
-            tag = f"{key}_{c['kind']}"
+            if c["fused"] and key == "topk":
+                continue
+            tag = ("index_topk" if c["fused"] and key == "index" else key) + f"_{c['kind']}"
             a = agg.setdefault(tag, {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0})
             a["ms"] += c[f"{key}_ms"]
             a["flops"] += c[key].get("flops", 0.0)
             a["bytes"] += c[key].get("bytes", 0.0)
             a["launches"] += 1
     dom_tag, dom = max(agg.items(), key=lambda kv: kv[1]["ms"])
-    if dom_tag in ("index_prefill", "attn_prefill"):
+    if dom_tag in ("index_prefill", "index_topk_prefill", "attn_prefill"):
         ach = dom["flops"] / (dom["ms"] / 1e3) / 1e12
         roof = {"kernel": dom_tag, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": None,

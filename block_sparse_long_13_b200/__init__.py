@@ -27,7 +27,7 @@ EXPORTS = (
     "msa_index_scores", "msa_topk_blocks", "msa_attn_prefill", "msa_attn_decode",
     "msa_prefill_workspace_bytes", "msa_decode_workspace_bytes", "msa_get_device_status",
     "msa_set_wait_limit_ns", "msa_debug_wait_timeout", "msa_status_string", "msa_last_error",
-    "msa_version", "msa_attn_decode_noalloc",
+    "msa_version", "msa_attn_decode_noalloc", "msa_index_topk",
 )
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, MSA_ERR_DEVICE_BOUNDS = range(6)
@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     sigs = {
         "msa_index_scores": [cfgp, batp, P, P, P, P],
         "msa_topk_blocks": [cfgp, batp, P, P, P],
+        "msa_index_topk": [cfgp, batp, P, P, P, P],
         "msa_attn_prefill": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
         "msa_attn_decode": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
         "msa_attn_decode_noalloc": [cfgp, batp, P, P, P, P, P, P, P],
@@ -184,6 +185,15 @@ def topk_blocks(cfg: Config, batch: Batch, block_scores, block_idx, stream=None)
     _check(lib.msa_topk_blocks(ctypes.byref(cfg._c()), ctypes.byref(batch._c()),
                                _need(block_scores, torch.float32, "block_scores"),
                                _need(block_idx, torch.int32, "block_idx"), _stream(stream)))
+
+
+def index_topk(cfg: Config, batch: Batch, idx_q, idx_k_cache, block_idx, stream=None) -> None:
+    """Indexer scores and top-k selection in one pass (the scores are not materialised)."""
+    lib = load_library()
+    _check(lib.msa_index_topk(ctypes.byref(cfg._c()), ctypes.byref(batch._c()),
+                              _need(idx_q, torch.bfloat16, "idx_q"),
+                              _need(idx_k_cache, torch.bfloat16, "idx_k_cache"),
+                              _need(block_idx, torch.int32, "block_idx"), _stream(stream)))
 
 
 def prefill_workspace_bytes(cfg: Config, batch: Batch) -> int:

@@ -16,7 +16,7 @@
 //
 // Roles: warp 0 = TMA producer (query tiles double-buffered, key tiles of a
 // (pair, head) through a ring), warp 1 = TMEM owner + single-thread UMMA
-// issuer, warps 2..5 / 6..9 = the two epilogue warpgroups.  Accumulators are
+// issuer, warps 4..7 / 8..11 = the two epilogue warpgroups.  Accumulators are
 // double-buffered (2 x 256 columns).  Units are dealt to persistent CTAs in a
 // snake order over a longest-first list, group-major so that one group's keys
 // are live in L2 at a time.
@@ -25,13 +25,21 @@
 
 namespace msa {
 
-constexpr int IDXP_THREADS = 320;
+constexpr int IDXP_THREADS = 384;   // warpgroup 0: producer + UMMA warps; warpgroups 1, 2: epilogue
+// Register split (setmaxnreg; registers are granted per warpgroup): the launch gives 168 per thread
+// (65536 / 384, rounded to 8); warpgroup 0 returns registers, the epilogue warpgroups take them.
+constexpr int IDXP_REGS_CTRL = 64, IDXP_REGS_EPI = 216;
+static_assert(128 * IDXP_REGS_CTRL + 256 * IDXP_REGS_EPI <= 384 * 168, "register split exceeds the launch");
 constexpr int IDXP_TILE = 128;
 constexpr int IDXP_MAXSEQ = 1024;
 constexpr int IDXP_STAGE_BYTES = 2 * IDXP_TILE * 64 * 2;   // keys of one head for two blocks: 32 KiB
 
+constexpr int IDXP_FUSED_SLOTS = 15;   // fused top-k: candidate slots per row (topk <= 16)
+
 struct IdxPrefillArgs {
-  float* scores;             // [total_q][Hkv][max_blocks]
+  float* scores;             // [total_q][Hkv][max_blocks] (score form)
+  int32_t* block_idx;        // [total_q][Hkv][topk] (fused form)
+  int topk;
   const int32_t* q_start;
   const int32_t* ctx_len;
   const int32_t* page_table;
@@ -44,6 +52,12 @@ struct IdxUnit {
   int qs, nq, ctx;
 };
 
+// FUSED = false: write every block score.  FUSED = true: keep, per row, the best topk-1 earlier blocks
+// by (score desc, block asc) in registers while the blocks stream by (each epilogue warpgroup sees
+// half of them), merge the two halves through shared memory at the end of the unit and write the
+// selection (ascending, the row's own block included, -1 padded): the same rule and the same fp32
+// scores as msa_topk_blocks, without materialising the score matrix.
+template <bool FUSED>
 __global__ void __launch_bounds__(IDXP_THREADS, 1)
 index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64, Hi, total_q), box (64, 1, 128)
                      const __grid_constant__ CUtensorMap tmap_k,   // idx_k  (64, 128, Hi, P), box (64, 128, 1, 1)
@@ -121,6 +135,8 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
     return true;
   };
 
+  if (warp < 4) {
+  regs_dec<IDXP_REGS_CTRL>();   // warps 2 and 3 have no role; they wait at the final barrier
   if (warp == 0) {
     // ------------------------------------------------------------ producer warp
     // lane 0 issues the copies; the whole warp reads the page ids of the next 32 blocks at once
@@ -224,9 +240,11 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0);
     }
-  } else if (warp >= 2) {
+  }
+  } else {
+    regs_inc<IDXP_REGS_EPI>();
     // ------------------------------------------------------------ epilogue warpgroups
-    const int w = (warp - 2) >> 2;             // this warpgroup pools block 2*pair + w of every step
+    const int w = (warp - 4) >> 2;             // this warpgroup pools block 2*pair + w of every step
     const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;         // row of the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -237,10 +255,31 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
       const bool valid = r < u.nrows;
       const int row = u.row0 + r;
       const int p = u.ctx - u.nq + (row - u.qs);
-      float* srow = a.scores + (static_cast<long>(row) * a.Hkv + u.g) * a.max_blocks;
+      float* srow = FUSED ? nullptr : a.scores + (static_cast<long>(row) * a.Hkv + u.g) * a.max_blocks;
       const int nstep = ((u.nblk + 1) >> 1) * a.hg;
       bool ok = true;
       float tot = 0.f;
+      // fused form: candidate keys (order_key(score) << 32 | ~block); unused slots hold ~0 and are never
+      // replaced, so kmin is the smallest key among the topk-1 live slots (0 = empty)
+      const int cur_blk = p >= 0 ? p / a.block_size : -1;
+      uint64_t ck[IDXP_FUSED_SLOTS];
+      uint64_t kmin = 0;
+      int kpos = 0;
+      if (FUSED) {
+#pragma unroll
+        for (int i = 0; i < IDXP_FUSED_SLOTS; ++i) ck[i] = i < a.topk - 1 ? 0ull : ~0ull;
+        kmin = a.topk > 1 ? 0ull : ~0ull;
+      }
+      auto insert = [&](uint64_t key) {          // replace the smallest live slot with key (key > kmin)
+#pragma unroll
+        for (int i = 0; i < IDXP_FUSED_SLOTS; ++i)
+          if (i == kpos) ck[i] = key;
+        kmin = ck[0];
+        kpos = 0;
+#pragma unroll
+        for (int i = 1; i < IDXP_FUSED_SLOTS; ++i)
+          if (ck[i] < kmin) { kmin = ck[i]; kpos = i; }
+      };
       for (int sp = 0; sp < nstep; ++sp, ++ait) {
         const int hl = sp % a.hg;
         const int b = 2 * (sp / a.hg) + w;     // this warpgroup's block
@@ -275,7 +314,55 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
         }
         const float hm = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], fmax3(mx[4], mx[5], mx[6]), mx[7]));
         tot = (hl == 0) ? hm : tot + hm;
-        if (hl == a.hg - 1 && valid && b < u.nblk) __stcs(srow + b, tot);  // -inf past the row's block
+        if (FUSED) {
+          if (hl == a.hg - 1 && valid && b < cur_blk && tot > -INFINITY) {   // candidates: earlier blocks
+            const uint64_t key = (static_cast<uint64_t>(order_key(tot)) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(b));
+            if (key > kmin) insert(key);
+          }
+        } else if (hl == a.hg - 1 && valid && b < u.nblk) {
+          __stcs(srow + b, tot);                 // -inf past the row's block
+        }
+      }
+      if (FUSED) {
+        // merge the two warpgroups' halves: warp (4 + quarter) and warp (8 + quarter) own the same rows
+        uint64_t* xb = reinterpret_cast<uint64_t*>(k_smem + a.stages * IDXP_STAGE_BYTES) + r * IDXP_FUSED_SLOTS;
+        if (w == 1) {
+#pragma unroll
+          for (int i = 0; i < IDXP_FUSED_SLOTS; ++i) xb[i] = ck[i];
+        }
+        if (named_bar_any(1 + quarter, 64, !ok)) break;   // both warps of the pair leave together
+        if (w == 0) {
+#pragma unroll
+          for (int i = 0; i < IDXP_FUSED_SLOTS; ++i) {
+            const uint64_t key = xb[i];
+            if (key != ~0ull && key > kmin) insert(key);
+          }
+        }
+        named_bar_sync(1 + quarter, 64);        // the partner may refill the buffer for its next unit
+        if (w == 0 && valid) {
+          int32_t* orow = a.block_idx + (static_cast<long>(row) * a.Hkv + u.g) * a.topk;
+          if (cur_blk < 0 || cur_blk >= a.max_blocks) {
+            flag_error(MSA_DEV_BOUNDS);
+            for (int j = 0; j < a.topk; ++j) orow[j] = -1;
+          } else {
+            int nsel = 0;
+#pragma unroll
+            for (int i = 0; i < IDXP_FUSED_SLOTS; ++i) nsel += (ck[i] != 0ull && ck[i] != ~0ull) ? 1 : 0;
+#pragma unroll
+            for (int i = 0; i < IDXP_FUSED_SLOTS; ++i) {
+              if (ck[i] != 0ull && ck[i] != ~0ull) {
+                const uint32_t bi = 0xFFFFFFFFu - static_cast<uint32_t>(ck[i]);
+                int rank = 0;                    // ids are distinct: rank = number of smaller ids
+#pragma unroll
+                for (int j = 0; j < IDXP_FUSED_SLOTS; ++j)
+                  rank += (ck[j] != 0ull && ck[j] != ~0ull && 0xFFFFFFFFu - static_cast<uint32_t>(ck[j]) < bi) ? 1 : 0;
+                orow[rank] = static_cast<int32_t>(bi);
+              }
+            }
+            orow[nsel] = cur_blk;                // every candidate lies before the row's own block
+            for (int j = nsel + 1; j < a.topk; ++j) orow[j] = -1;
+          }
+        }
       }
       if (!ok) break;
     }

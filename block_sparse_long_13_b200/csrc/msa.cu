@@ -203,6 +203,56 @@ __global__ void wait_forever_probe_kernel() {
 
 }  // namespace
 
+// Tensor-core indexer (any batch shape; the streaming form is faster for few queries per sequence).
+template <bool FUSED>
+msa_status_t launch_index_prefill(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
+                                  const void* idx_k_cache, float* block_scores, int32_t* block_idx,
+                                  cudaStream_t stream) {
+  msa_status_t st;
+  const int Hi = cfg->idx_heads, Hkv = cfg->num_kv_heads, hg = Hi / Hkv;
+  const int sms = num_sms();
+  CHECK_SUP(batch->num_seqs <= msa::IDXP_MAXSEQ, "at most %d sequences per tensor-core indexer call",
+            msa::IDXP_MAXSEQ);
+  CUtensorMap tk;
+  {
+    const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
+    const uint64_t strides[3] = {128, 128 * 128, static_cast<uint64_t>(Hi) * 128 * 128};
+    const uint32_t box[4] = {64, 128, 1, 1};
+    if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box)) != MSA_OK) return st;
+  }
+  CUtensorMap tq;
+  {
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->total_q)};
+    const uint64_t strides[2] = {128, static_cast<uint64_t>(Hi) * 128};
+    const uint32_t box[3] = {64, 1, 128};
+    if ((st = make_map(&tq, idx_q, 3, dims, strides, box)) != MSA_OK) return st;
+  }
+  msa::IdxPrefillArgs a{};
+  a.scores = block_scores;
+  a.block_idx = block_idx;
+  a.topk = cfg->topk;
+  a.q_start = batch->q_start;
+  a.ctx_len = batch->ctx_len;
+  a.page_table = batch->page_table;
+  a.num_seqs = batch->num_seqs;
+  a.total_q = batch->total_q;
+  a.max_blocks = batch->max_blocks_per_seq;
+  a.num_pages = batch->num_pages;
+  a.Hi = Hi;
+  a.Hkv = Hkv;
+  a.hg = hg;
+  a.block_size = cfg->block_size;
+  const int q_tile = hg * 128 * 64 * 2;
+  const int xbuf = FUSED ? 128 * msa::IDXP_FUSED_SLOTS * 8 : 0;   // candidate exchange between warpgroups
+  a.nqbuf = (2 * q_tile + 2 * msa::IDXP_STAGE_BYTES <= 200 * 1024 - xbuf) ? 2 : 1;
+  a.stages = std::min(8, (200 * 1024 - xbuf - a.nqbuf * q_tile) / msa::IDXP_STAGE_BYTES);
+  CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
+  const int smem = a.nqbuf * q_tile + a.stages * msa::IDXP_STAGE_BYTES + xbuf + 1024;
+  CUDA_TRY(set_smem(msa::index_prefill_kernel<FUSED>, smem));
+  msa::index_prefill_kernel<FUSED><<<sms, msa::IDXP_THREADS, smem, stream>>>(tq, tk, a);
+  return launched();
+}
+
 extern "C" {
 
 const char* msa_status_string(msa_status_t s) {
@@ -240,15 +290,15 @@ msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch,
   CHECK_ARG(aligned16(idx_q) && aligned16(idx_k_cache) && aligned16(block_scores), "pointers must be 16-byte aligned");
   if (batch->total_q == 0) return MSA_OK;
   const int Hi = cfg->idx_heads, Hkv = cfg->num_kv_heads, hg = Hi / Hkv;
-  CUtensorMap tk;
-  {
-    const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
-    const uint64_t strides[3] = {128, 128 * 128, static_cast<uint64_t>(Hi) * 128 * 128};
-    const uint32_t box[4] = {64, 128, static_cast<uint32_t>(hg), 1};
-    if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box)) != MSA_OK) return st;
-  }
-  const int sms = num_sms();
   if (batch->max_q_per_seq <= msa::IDXD_MAXQ) {
+    CUtensorMap tk;
+    {
+      const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
+      const uint64_t strides[3] = {128, 128 * 128, static_cast<uint64_t>(Hi) * 128 * 128};
+      const uint32_t box[4] = {64, 128, static_cast<uint32_t>(hg), 1};
+      if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box)) != MSA_OK) return st;
+    }
+    const int sms = num_sms();
     CHECK_SUP(batch->num_seqs <= msa::IDXD_MAXSEQ, "at most %d sequences per streaming indexer call",
               msa::IDXD_MAXSEQ);
     msa::IdxDecodeArgs a{};
@@ -281,42 +331,7 @@ msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch,
     if (mq <= 4) return go(msa::index_decode_kernel<4>);
     return go(msa::index_decode_kernel<8>);
   }
-  CHECK_SUP(batch->num_seqs <= msa::IDXP_MAXSEQ, "at most %d sequences per tensor-core indexer call",
-            msa::IDXP_MAXSEQ);
-  {
-    const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
-    const uint64_t strides[3] = {128, 128 * 128, static_cast<uint64_t>(Hi) * 128 * 128};
-    const uint32_t box[4] = {64, 128, 1, 1};
-    if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box)) != MSA_OK) return st;
-  }
-  CUtensorMap tq;
-  {
-    const uint64_t dims[3] = {64, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->total_q)};
-    const uint64_t strides[2] = {128, static_cast<uint64_t>(Hi) * 128};
-    const uint32_t box[3] = {64, 1, 128};
-    if ((st = make_map(&tq, idx_q, 3, dims, strides, box)) != MSA_OK) return st;
-  }
-  msa::IdxPrefillArgs a{};
-  a.scores = block_scores;
-  a.q_start = batch->q_start;
-  a.ctx_len = batch->ctx_len;
-  a.page_table = batch->page_table;
-  a.num_seqs = batch->num_seqs;
-  a.total_q = batch->total_q;
-  a.max_blocks = batch->max_blocks_per_seq;
-  a.num_pages = batch->num_pages;
-  a.Hi = Hi;
-  a.Hkv = Hkv;
-  a.hg = hg;
-  a.block_size = cfg->block_size;
-  const int q_tile = hg * 128 * 64 * 2;
-  a.nqbuf = (2 * q_tile + 2 * msa::IDXP_STAGE_BYTES <= 200 * 1024) ? 2 : 1;
-  a.stages = std::min(8, (200 * 1024 - a.nqbuf * q_tile) / msa::IDXP_STAGE_BYTES);
-  CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
-  const int smem = a.nqbuf * q_tile + a.stages * msa::IDXP_STAGE_BYTES + 1024;
-  CUDA_TRY(set_smem(msa::index_prefill_kernel, smem));
-  msa::index_prefill_kernel<<<sms, msa::IDXP_THREADS, smem, stream>>>(tq, tk, a);
-  return launched();
+  return launch_index_prefill<false>(cfg, batch, idx_q, idx_k_cache, block_scores, nullptr, stream);
 }
 
 msa_status_t msa_topk_blocks(const msa_config_t* cfg, const msa_batch_t* batch, const float* block_scores,
@@ -345,6 +360,19 @@ msa_status_t msa_topk_blocks(const msa_config_t* cfg, const msa_batch_t* batch, 
   }
 #undef TOPK_ARGS
   return launched();
+}
+
+msa_status_t msa_index_topk(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
+                            const void* idx_k_cache, int32_t* block_idx, cudaStream_t stream) {
+  msa_status_t st;
+  if ((st = check_config(cfg)) != MSA_OK) return st;
+  if ((st = check_batch(batch)) != MSA_OK) return st;
+  CHECK_ARG(idx_q && idx_k_cache && block_idx, "idx_q, idx_k_cache and block_idx must not be NULL");
+  CHECK_ARG(aligned16(idx_q) && aligned16(idx_k_cache) && aligned16(block_idx), "pointers must be 16-byte aligned");
+  CHECK_SUP(cfg->topk <= msa::IDXP_FUSED_SLOTS + 1, "the fused indexer keeps at most %d blocks per row",
+            msa::IDXP_FUSED_SLOTS + 1);
+  if (batch->total_q == 0) return MSA_OK;
+  return launch_index_prefill<true>(cfg, batch, idx_q, idx_k_cache, nullptr, block_idx, stream);
 }
 
 msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch, const void* q, const void* k_cache,

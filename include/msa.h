@@ -126,6 +126,23 @@ msa_status_t msa_topk_blocks(const msa_config_t* cfg, const msa_batch_t* batch, 
                              int32_t* block_idx, cudaStream_t stream);
 
 /*
+ * msa_index_scores followed by msa_topk_blocks in one pass, without the score
+ * matrix: while a row's key blocks stream through the tensor-core indexer, its
+ * best topk-1 earlier blocks are kept on chip by the same (score desc, block
+ * asc) rule, from the same fp32 scores, so block_idx is identical to the
+ * two-call result.  (24-ai.news: each query group scores all blocks with
+ * light indexer score kernels and keeps only the most relevant; inteligile
+ * "MiniMax-M3" model page, tag "Exp-free TopK kernel".  The pages do not say
+ * whether the two are fused; this call is this library's fused form.)
+ * block_idx: int32 [total_q][num_kv_heads][topk].
+ * Requires topk <= 16 (MSA_ERR_UNSUPPORTED otherwise).  Always runs the
+ * tensor-core form; batches with few queries per sequence are better served
+ * by the two calls.
+ */
+msa_status_t msa_index_topk(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
+                            const void* idx_k_cache, int32_t* block_idx, cudaStream_t stream);
+
+/*
  * Sparse GQA attention, block-major ("KV outer, gather Q": shaam.blog,
  * section "What makes MiniMax M3 different ..."; daily.dev, "Serving
  * options": KV-block-major prefill scheduling).  Query head h of row t uses

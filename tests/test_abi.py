@@ -106,6 +106,21 @@ def test_bad_batch_and_pointers_rejected(lib):
     assert lib.msa_set_wait_limit_ns(0) == msa.MSA_ERR_INVALID_ARG
 
 
+def test_fused_index_topk_checks(lib):
+    """The fused call validates like the two calls it replaces and keeps at most 16 blocks per row."""
+    b = _batch()._c(host_only=True)
+    p = ctypes.c_void_p(16)
+    cfg17 = _cfg(topk=17)._c()
+    assert lib.msa_index_topk(ctypes.byref(cfg17), ctypes.byref(b), p, p, p, None) == msa.MSA_ERR_UNSUPPORTED
+    assert b"16" in lib.msa_last_error()
+    cfg = msa.Config()._c()
+    assert lib.msa_index_topk(ctypes.byref(cfg), ctypes.byref(b), p, None, p, None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_index_topk(ctypes.byref(cfg), ctypes.byref(b), p, p, ctypes.c_void_p(20), None) == \
+        msa.MSA_ERR_INVALID_ARG
+    bad = _cfg(head_dim=64)._c()
+    assert lib.msa_index_topk(ctypes.byref(bad), ctypes.byref(b), p, p, p, None) == msa.MSA_ERR_UNSUPPORTED
+
+
 def test_workspace_sizes_scale_with_the_batch(lib):
     cfg = msa.Config()
     b1 = msa.Batch.make([0, 16384], [16384], [list(range(128))], 128, device="cpu")
