@@ -51,6 +51,24 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu record (profiles/traffic.json), or
+    None when there is none or the kernel's sources changed since it was taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for rel in rec["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return rec["dram_bytes_per_launch"] if h.hexdigest() == rec["sources_sha256"] else None
+
+
 # ------------------------------------------------------------------ workload parts
 
 class Part:
@@ -99,8 +117,13 @@ class Part:
             ev[2].record(stream)
         if stop_after == "attn":
             fn = m.attn_prefill if self.kind == "prefill" else m.attn_decode
+            phases = ev is not None and self.kind == "prefill"
+            if phases:
+                m.set_timing_events(ev[4:8])
             fn(self.cfg, self.batch, self.q, self.caches["k"], self.caches["v"], self.sel, self.out, self.lse,
                ws[:self.ws_bytes])
+            if phases:
+                m.set_timing_events(None)
         if ev is not None:
             ev[3].record(stream)
 
@@ -124,6 +147,13 @@ class Part:
         flops = keys * G * 4 * wl.head_dim
         bytes_ = keys * 2 * wl.head_dim * 2 + self.q.numel() * 2 * 2
         return {"flops": flops, "bytes": bytes_}
+
+    def merge_work(self):
+        """Partial O (bf16) and lse of every valid slot read once; out and lse written."""
+        wl = self.wl
+        slots = float((self.sel >= 0).sum())
+        G = wl.num_q_heads // wl.num_kv_heads
+        return {"bytes": slots * G * (wl.head_dim * 2 + 4) + wl.total_q * wl.num_q_heads * (wl.head_dim * 2 + 4)}
 
     def topk_work(self):
         cur = (self.pos // self.wl.block_size).double()
@@ -355,7 +385,8 @@ def main():
     if st != msa.MSA_OK:
         raise SystemExit(f"device status {st} after warm-up")
 
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nev)]
+    # per step and part: 4 call boundaries, then (prefill) the 4 phase events of msa_attn_prefill
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(nev)]
            for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
@@ -380,44 +411,71 @@ def main():
         t_idx = statistics.mean(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps))
         t_top = statistics.mean(evs[k][i][1].elapsed_time(evs[k][i][2]) for k in range(args.steps))
         t_att = statistics.mean(evs[k][i][2].elapsed_time(evs[k][i][3]) for k in range(args.steps))
-        calls[p.name] = {"index_ms": t_idx, "topk_ms": t_top, "attn_ms": t_att,
+        phase = None
+        if p.kind == "prefill" and args.stop_after == "attn":
+            phase = {nm: statistics.mean(evs[k][i][4 + j].elapsed_time(evs[k][i][5 + j]) for k in range(args.steps))
+                     for j, nm in enumerate(("schedule_ms", "kernel_ms", "merge_ms"))}
+        calls[p.name] = {"index_ms": t_idx, "topk_ms": t_top, "attn_ms": t_att, "attn_phases": phase,
                          "index": p.index_work(), "attn": p.attn_work(), "topk": p.topk_work(), "kind": p.kind,
+                         "merge": p.merge_work() if p.kind == "prefill" else None,
                          "tokens": p.wl.total_q, "fused": p.fused}
     pk = peaks()
-    # dominant call type over the step
-    agg = {}
-    for name, c in calls.items():
-        for key in ("index", "topk", "attn"):
-            if c["fused"] and key == "topk":
-                continue
-            tag = ("index_topk" if c["fused"] and key == "index" else key) + f"_{c['kind']}"
-            a = agg.setdefault(tag, {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0})
-            a["ms"] += c[f"{key}_ms"]
-            a["flops"] += c[key].get("flops", 0.0)
-            a["bytes"] += c[key].get("bytes", 0.0)
-            a["launches"] += 1
-    dom_tag, dom = max(agg.items(), key=lambda kv: kv[1]["ms"])
-    if dom_tag in ("index_prefill", "index_topk_prefill", "attn_prefill"):
-        ach = dom["flops"] / (dom["ms"] / 1e3) / 1e12
-        roof = {"kernel": dom_tag, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": None,
-                "peak_source": pk["source"] + " (burst bf16)", "launch_ms": dom["ms"] / dom["launches"]}
-    else:
-        ach = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
-        roof = {"kernel": dom_tag, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"] + " (copy)",
-                "launch_ms": dom["ms"] / dom["launches"]}
-    fractions = {}
-    for tag, a in agg.items():
-        if a["ms"] <= 0:
-            continue
-        if "prefill" in tag and tag != "topk_prefill":
-            fractions[tag] = {"tflops": a["flops"] / a["ms"] / 1e9, "frac_of_measured_bf16":
-                              a["flops"] / a["ms"] / 1e9 / pk["bf16_tflops"], "ms_per_step": a["ms"]}
+    # per kernel: device time per step (CUDA events on the launching stream) and algorithmic work
+    kern = {}
+
+    def addk(name, ms, launches, flops=0.0, bytes_=0.0):
+        k = kern.setdefault(name, {"ms": 0.0, "launches": 0, "flops": 0.0, "bytes": 0.0})
+        k["ms"] += ms
+        k["launches"] += launches
+        k["flops"] += flops
+        k["bytes"] += bytes_
+
+    for c in calls.values():
+        if c["kind"] == "prefill":
+            if c["fused"]:
+                addk("index_prefill_kernel (fused top-k)", c["index_ms"], 1, flops=c["index"]["flops"])
+            else:
+                addk("index_prefill_kernel", c["index_ms"], 1, flops=c["index"]["flops"])
+                addk("topk_blocks_kernel (prefill)", c["topk_ms"], 1, bytes_=c["topk"]["bytes"])
+            ph = c["attn_phases"]
+            if ph is not None:
+                addk("schedule (4 kernels)", ph["schedule_ms"], 4)
+                addk("attn_prefill_kernel", ph["kernel_ms"], 1, flops=c["attn"]["flops"])
+                addk("attn_merge_kernel", ph["merge_ms"], 1, bytes_=c["merge"]["bytes"])
         else:
-            gbs = a["bytes"] / a["ms"] / 1e6
-            fractions[tag] = {"gbs": gbs, "frac_of_measured_hbm": gbs / pk["hbm_gbs"],
-                              "frac_of_8tbs": gbs / 8000.0, "ms_per_step": a["ms"]}
+            addk("index_decode_kernel", c["index_ms"], 1, bytes_=c["index"]["bytes"])
+            addk("topk_blocks_kernel (decode)", c["topk_ms"], 1, bytes_=c["topk"]["bytes"])
+            addk("attn_decode_kernel", c["attn_ms"], 1, bytes_=c["attn"]["bytes"])
+    # every kernel is timed inside a step of tens of ms: the sustained tensor peak is the denominator
+    tensor_peak, tensor_src = pk["bf16_tflops_sustained"], pk["source"] + " sustained bf16 (cuBLAS, power-capped)"
+    fractions = {}
+    for name, k in kern.items():
+        if k["ms"] <= 0:
+            continue
+        if k["flops"] > 0:
+            ach = k["flops"] / k["ms"] / 1e9
+            fractions[name] = {"ms_per_step": k["ms"], "launches_per_step": k["launches"], "tflops": ach,
+                               "frac": ach / tensor_peak}
+        elif k["bytes"] > 0:
+            ach = k["bytes"] / k["ms"] / 1e6
+            fractions[name] = {"ms_per_step": k["ms"], "launches_per_step": k["launches"], "gbs": ach,
+                               "frac": ach / pk["hbm_gbs"]}
+        else:
+            fractions[name] = {"ms_per_step": k["ms"], "launches_per_step": k["launches"]}
+    dom_name, dom = max(((n, k) for n, k in kern.items() if k["flops"] > 0 or k["bytes"] > 0),
+                        key=lambda nk: nk[1]["ms"])
+    launch_ms = dom["ms"] / dom["launches"]
+    traffic = recorded_traffic(dom_name)
+    if dom["flops"] > 0:
+        ach = dom["flops"] / dom["launches"] / (launch_ms / 1e3) / 1e12
+        roof = {"kernel": dom_name, "bound": "tensor", "achieved": ach, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": ach / tensor_peak, "traffic": traffic, "peak_source": tensor_src, "launch_ms": launch_ms,
+                "flops_per_launch": dom["flops"] / dom["launches"]}
+    else:
+        ach = dom["bytes"] / dom["launches"] / (launch_ms / 1e3) / 1e9
+        roof = {"kernel": dom_name, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "traffic": traffic, "peak_source": pk["source"] + " copy",
+                "launch_ms": launch_ms, "bytes_per_launch": dom["bytes"] / dom["launches"]}
     parts_summary = {}
     pre = [c for c in calls.values() if c["kind"] == "prefill"]
     if pre:

@@ -27,7 +27,7 @@ EXPORTS = (
     "msa_index_scores", "msa_topk_blocks", "msa_attn_prefill", "msa_attn_decode",
     "msa_prefill_workspace_bytes", "msa_decode_workspace_bytes", "msa_get_device_status",
     "msa_set_wait_limit_ns", "msa_debug_wait_timeout", "msa_status_string", "msa_last_error",
-    "msa_version", "msa_attn_decode_noalloc", "msa_index_topk",
+    "msa_version", "msa_attn_decode_noalloc", "msa_index_topk", "msa_set_timing_events",
 )
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, MSA_ERR_DEVICE_BOUNDS = range(6)
@@ -70,6 +70,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "msa_index_scores": [cfgp, batp, P, P, P, P],
         "msa_topk_blocks": [cfgp, batp, P, P, P],
         "msa_index_topk": [cfgp, batp, P, P, P, P],
+        "msa_set_timing_events": [P, ctypes.c_int32],
         "msa_attn_prefill": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
         "msa_attn_decode": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
         "msa_attn_decode_noalloc": [cfgp, batp, P, P, P, P, P, P, P],
@@ -194,6 +195,21 @@ def index_topk(cfg: Config, batch: Batch, idx_q, idx_k_cache, block_idx, stream=
                               _need(idx_q, torch.bfloat16, "idx_q"),
                               _need(idx_k_cache, torch.bfloat16, "idx_k_cache"),
                               _need(block_idx, torch.int32, "block_idx"), _stream(stream)))
+
+
+def set_timing_events(events=None) -> None:
+    """Record four torch.cuda.Event (created with enable_timing=True) around the phases of the
+    following msa_attn_prefill calls on this thread: schedule, block-major kernel, merge.
+    None stops recording."""
+    lib = load_library()
+    if not events:
+        _check(lib.msa_set_timing_events(None, 0))
+        return
+    for e in events:
+        if not e.cuda_event:     # torch creates the CUDA event on its first record
+            e.record()
+    handles = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib.msa_set_timing_events(handles, 4))
 
 
 def prefill_workspace_bytes(cfg: Config, batch: Batch) -> int:

@@ -21,6 +21,12 @@ namespace {
 
 thread_local char g_msg[512] = "";
 
+// optional phase events of msa_attn_prefill on this host thread (msa_set_timing_events)
+thread_local cudaEvent_t g_phase_ev[4] = {nullptr, nullptr, nullptr, nullptr};
+inline void phase_mark(int i, cudaStream_t stream) {
+  if (g_phase_ev[i]) cudaEventRecord(g_phase_ev[i], stream);
+}
+
 msa_status_t fail(msa_status_t st, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -412,6 +418,7 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
   s.page_table = batch->page_table;
   s.num_pages = batch->num_pages;
   s.max_tiles = static_cast<int>(w.max_tiles);
+  phase_mark(0, stream);
   CUDA_TRY(cudaMemsetAsync(s.counts, 0, w.nbuckets * 4, stream));
   const unsigned sgrid = static_cast<unsigned>((batch->total_q + msa::SCHED_ROWS - 1) / msa::SCHED_ROWS);
   msa::sched_count_scatter_kernel<<<sgrid, 256, 0, stream>>>(s, 0);
@@ -454,8 +461,10 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
   a.max_tiles = s.max_tiles;
   a.scale_log2 = softmax_scale(cfg) * 1.4426950408889634f;
   CUDA_TRY(set_smem(msa::attn_prefill_kernel, msa::ATTP_SMEM));
+  phase_mark(1, stream);
   msa::attn_prefill_kernel<<<sms, msa::ATTP_THREADS, msa::ATTP_SMEM, stream>>>(tq, tk, tv, tpo, a);
   if ((st = launched()) != MSA_OK) return st;
+  phase_mark(2, stream);
 
   msa::MergeArgs m{};
   m.part_o = reinterpret_cast<const __nv_bfloat16*>(ws + w.part_o);
@@ -468,7 +477,15 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
   m.Hkv = Hkv;
   m.topk = k;
   msa::attn_merge_kernel<<<static_cast<unsigned>(batch->total_q) * Hkv, 256, 0, stream>>>(m);
-  return launched();
+  if ((st = launched()) != MSA_OK) return st;
+  phase_mark(3, stream);
+  return MSA_OK;
+}
+
+msa_status_t msa_set_timing_events(void* const* events, int32_t n) {
+  CHECK_ARG(n == 0 || (n == 4 && events != nullptr), "pass 4 events, or 0 to stop recording");
+  for (int i = 0; i < 4; ++i) g_phase_ev[i] = n ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+  return MSA_OK;
 }
 
 msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, const void* q, const void* k_cache,

@@ -193,6 +193,14 @@ msa_status_t msa_attn_decode_noalloc(const msa_config_t* cfg, const msa_batch_t*
                                      const void* k_cache, const void* v_cache, const int32_t* block_idx, void* out,
                                      float* lse, cudaStream_t stream);
 
+/* Timing hook (no counterpart on the pages).  With n = 4 and four cudaEvent_t
+ * handles (owned by the caller), every later msa_attn_prefill call on this host
+ * thread records events[0] before its schedule kernels, events[1] before the
+ * block-major attention kernel, events[2] after it and events[3] after the
+ * merge, on its stream, so the phases can be timed with cudaEventElapsedTime.
+ * n = 0 stops recording.  Any other n is MSA_ERR_INVALID_ARG. */
+msa_status_t msa_set_timing_events(void* const* events, int32_t n);
+
 /* Workspace sizes (bytes) for the two attention calls; only the host fields of
  * `batch` are read.  0 means the arguments are invalid. */
 size_t msa_prefill_workspace_bytes(const msa_config_t* cfg, const msa_batch_t* batch);

@@ -121,6 +121,12 @@ def test_fused_index_topk_checks(lib):
     assert lib.msa_index_topk(ctypes.byref(bad), ctypes.byref(b), p, p, p, None) == msa.MSA_ERR_UNSUPPORTED
 
 
+def test_timing_events_hook_checks(lib):
+    assert lib.msa_set_timing_events(None, 3) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_set_timing_events(None, 4) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_set_timing_events(None, 0) == msa.MSA_OK
+
+
 def test_workspace_sizes_scale_with_the_batch(lib):
     cfg = msa.Config()
     b1 = msa.Batch.make([0, 16384], [16384], [list(range(128))], 128, device="cpu")
