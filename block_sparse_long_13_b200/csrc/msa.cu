@@ -352,9 +352,9 @@ msa_status_t msa_topk_blocks(const msa_config_t* cfg, const msa_batch_t* batch, 
   const int Hkv = cfg->num_kv_heads, k = cfg->topk, bs = cfg->block_size;
 #define TOPK_ARGS block_scores, block_idx, batch->q_start, batch->ctx_len, batch->num_seqs, batch->total_q, Hkv, nb, k, bs
   if (nb <= 256) {
-    msa::topk_blocks_kernel<1, 8><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(TOPK_ARGS);
+    msa::topk_row_warp_kernel<8><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(TOPK_ARGS);
   } else if (nb <= 1024) {
-    msa::topk_blocks_kernel<1, 32><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(TOPK_ARGS);
+    msa::topk_row_warp_kernel<32><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(TOPK_ARGS);
   } else if (nb <= 2048) {
     msa::topk_blocks_kernel<2, 32><<<static_cast<unsigned>(rows), 64, 0, stream>>>(TOPK_ARGS);
   } else if (nb <= 4096) {

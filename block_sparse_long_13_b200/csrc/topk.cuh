@@ -37,8 +37,6 @@ topk_blocks_kernel(const float* __restrict__ scores, int32_t* __restrict__ out,
   __shared__ int s_cnt[W > 1 ? W : 1];
   __shared__ int s_sel[W > 1 ? 64 : 1];
   __shared__ int s_nsel;
-  __shared__ uint64_t s_cand[W == 1 ? 4 : 1][64];   // fast-path candidates, one area per warp
-  __shared__ uint64_t s_thr[W == 1 ? 4 : 1];
   if (row >= nrows) return;  // W == 1: whole warp leaves together; W > 1: whole CTA
   const int tid = (W == 1) ? lane : static_cast<int>(threadIdx.x);
   const int t = static_cast<int>(row / Hkv);
@@ -86,54 +84,7 @@ topk_blocks_kernel(const float* __restrict__ scores, int32_t* __restrict__ out,
   const int total_valid = block_sum(nvalid);
   const bool take_all = total_valid <= m;
   uint64_t thr = 1;  // keep valid keys >= thr
-  bool found = false;
-  if (W == 1 && !take_all && m > 0 && m <= 32) {
-    // Fast path.  The m-th largest of the 32 lane maxima bounds the m-th
-    // largest key from below (those m lane maxima are m distinct keys), so the
-    // answer is among the few keys at or above it: rank those exactly.
-    uint64_t lmax = 0;
-#pragma unroll
-    for (int i = 0; i < NPER; ++i) lmax = key[i] > lmax ? key[i] : lmax;
-    uint64_t lo = 0;
-    for (int bit = 63; bit >= 0; --bit) {
-      const uint64_t probe = lo | (1ull << bit);
-      const int c = __popc(__ballot_sync(0xFFFFFFFFu, lmax >= probe));
-      if (c >= m) {
-        lo = probe;
-        if (c == m) break;
-      }
-    }
-    if (lo != 0) {
-      int cl = 0;
-#pragma unroll
-      for (int i = 0; i < NPER; ++i) cl += (key[i] >= lo) ? 1 : 0;
-      int incl = cl;  // inclusive prefix over lanes
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += n;
-      }
-      const int ncand = __shfl_sync(0xFFFFFFFFu, incl, 31);
-      if (ncand <= 64) {
-        uint64_t* cand = s_cand[warp];
-        int at = incl - cl;
-#pragma unroll
-        for (int i = 0; i < NPER; ++i)
-          if (key[i] >= lo) cand[at++] = key[i];
-        __syncwarp();
-        for (int c = lane; c < ncand; c += 32) {
-          const uint64_t kc = cand[c];
-          int above = 0;
-          for (int d = 0; d < ncand; ++d) above += (cand[d] > kc) ? 1 : 0;
-          if (above == m - 1) s_thr[warp] = kc;   // exactly one candidate: keys are distinct
-        }
-        __syncwarp();
-        thr = s_thr[warp];
-        found = true;
-      }
-    }
-  }
-  if (!take_all && m > 0 && !found) {
+  if (!take_all && m > 0) {
     uint64_t prefix = 0;
     for (int bit = 63; bit >= 0; --bit) {
       const uint64_t probe = prefix | (1ull << bit);
@@ -183,6 +134,147 @@ topk_blocks_kernel(const float* __restrict__ scores, int32_t* __restrict__ out,
       for (int j = n + lane; j < topk; j += 32) orow[j] = (j == n) ? cur : -1;
     }
   }
+}
+
+
+// One warp per (row, group) for rows of up to 32 * NPER candidates.  Scores are
+// compared as 32-bit order-preserving keys; ties are broken by the lower block
+// id only where they matter.  The (topk-1)-th largest of the 32 lane maxima
+// bounds the threshold from below, so the answer lies among the few candidates
+// at or above it; those are ranked exactly, and the selected ids are sorted by
+// id for the output.  Rows where that set is large (or topk-1 > 32) take the
+// MSB-first bitwise search on 64-bit keys.
+template <int NPER>
+__global__ void __launch_bounds__(128) topk_row_warp_kernel(const float* __restrict__ scores, int32_t* __restrict__ out,
+                                                            const int32_t* __restrict__ q_start,
+                                                            const int32_t* __restrict__ ctx_len, int num_seqs,
+                                                            int total_q, int Hkv, int max_blocks, int topk,
+                                                            int block_size) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long row = static_cast<long>(blockIdx.x) * 4 + warp;
+  __shared__ uint32_t s_ck[4][64];
+  __shared__ int s_cb[4][64];
+  __shared__ int s_sel[4][64];
+  if (row >= static_cast<long>(total_q) * Hkv) return;   // whole warp
+  const int t = static_cast<int>(row / Hkv);
+  const int s = find_seq(q_start, num_seqs, t);
+  const int qs = __ldg(q_start + s);
+  const int nq = __ldg(q_start + s + 1) - qs;
+  const long p = static_cast<long>(__ldg(ctx_len + s)) - nq + (t - qs);
+  int32_t* orow = out + row * topk;
+  if (p < 0 || p / block_size >= max_blocks) {
+    if (lane == 0) flag_error(MSA_DEV_BOUNDS);
+    for (int j = lane; j < topk; j += 32) orow[j] = -1;
+    return;
+  }
+  const int cur = static_cast<int>(p / block_size);
+  const float* srow = scores + row * static_cast<long>(max_blocks);
+  // every load issued before any use (clamped in-bounds address where b >= cur)
+  float sv[NPER];
+  const int last = cur > 0 ? cur - 1 : 0;
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) sv[i] = __ldcs(srow + min(lane + i * 32, last));
+  uint32_t sk[NPER];   // order key of a finite candidate score (> 0), 0 otherwise
+  int nvalid = 0;
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) {
+    const bool ok = lane + i * 32 < cur && sv[i] > -INFINITY;   // excludes -inf and NaN
+    sk[i] = ok ? order_key(sv[i]) : 0u;
+    nvalid += ok ? 1 : 0;
+  }
+  const int m = topk - 1;   // free slots besides the current block
+  const int total = __reduce_add_sync(0xFFFFFFFFu, nvalid);
+  bool done = false;
+  if (total > m && m > 0 && m <= 32) {
+    uint32_t lmax = 0;
+#pragma unroll
+    for (int i = 0; i < NPER; ++i) lmax = max(lmax, sk[i]);
+    uint32_t lo = 0;   // count(lane maxima >= lo) >= m
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t probe = lo | (1u << bit);
+      const int c = __popc(__ballot_sync(0xFFFFFFFFu, lmax >= probe));
+      if (c >= m) {
+        lo = probe;
+        if (c == m) break;
+      }
+    }
+    if (lo != 0) {
+      int cl = 0;
+#pragma unroll
+      for (int i = 0; i < NPER; ++i) cl += sk[i] >= lo ? 1 : 0;
+      int incl = cl;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      const int ncand = __shfl_sync(0xFFFFFFFFu, incl, 31);
+      if (ncand <= 64) {
+        int at = incl - cl;
+#pragma unroll
+        for (int i = 0; i < NPER; ++i) {
+          if (sk[i] >= lo) {
+            s_ck[warp][at] = sk[i];
+            s_cb[warp][at] = lane + i * 32;
+            ++at;
+          }
+        }
+        __syncwarp();
+        // rank by (score desc, id asc); the first m are the selection
+        for (int c = lane; c < ncand; c += 32) {
+          const uint32_t kc = s_ck[warp][c];
+          const int bc = s_cb[warp][c];
+          int rank = 0;
+          for (int d = 0; d < ncand; ++d) {
+            const uint32_t kd = s_ck[warp][d];
+            rank += (kd > kc || (kd == kc && s_cb[warp][d] < bc)) ? 1 : 0;
+          }
+          if (rank < m) s_sel[warp][rank] = bc;
+        }
+        __syncwarp();
+        // ids ascending, then the row's own block (every candidate lies before it)
+        for (int j = lane; j < m; j += 32) {
+          const int b = s_sel[warp][j];
+          int r = 0;
+          for (int k = 0; k < m; ++k) r += s_sel[warp][k] < b ? 1 : 0;
+          orow[r] = b;
+        }
+        if (lane == 0) orow[m] = cur;
+        done = true;
+      }
+    }
+  }
+  if (done) return;
+  // general case: keep every candidate at or above the (m-th largest) 64-bit key
+  uint64_t thr = 1;
+  if (total > m && m > 0) {
+    uint64_t prefix = 0;
+    for (int bit = 63; bit >= 0; --bit) {
+      const uint64_t probe = prefix | (1ull << bit);
+      int c = 0;
+#pragma unroll
+      for (int i = 0; i < NPER; ++i) {
+        const uint64_t key = sk[i] ? (static_cast<uint64_t>(sk[i]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(lane + i * 32)) : 0ull;
+        c += key >= probe ? 1 : 0;
+      }
+      const int tot = __reduce_add_sync(0xFFFFFFFFu, c);
+      if (tot >= m) {
+        prefix = probe;
+        if (tot == m) break;   // keys are distinct
+      }
+    }
+    thr = prefix;
+  }
+  int base = 0;
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) {
+    const uint64_t key = sk[i] ? (static_cast<uint64_t>(sk[i]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(lane + i * 32)) : 0ull;
+    const bool sel = m > 0 && key != 0 && key >= thr;
+    const unsigned msk = __ballot_sync(0xFFFFFFFFu, sel);
+    if (sel) orow[base + __popc(msk & ((1u << lane) - 1u))] = lane + i * 32;
+    base += __popc(msk);
+  }
+  for (int j = base + lane; j < topk; j += 32) orow[j] = (j == base) ? cur : -1;
 }
 
 }  // namespace msa
