@@ -60,7 +60,7 @@ struct IdxUnit {
 template <bool FUSED>
 __global__ void __launch_bounds__(IDXP_THREADS, 1)
 index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64, Hi, total_q), box (64, 1, 128)
-                     const __grid_constant__ CUtensorMap tmap_k,   // idx_k  (64, 128, Hi, P), box (64, 128, 1, 1)
+                     const __grid_constant__ CUtensorMap tmap_k,   // idx_k  (64, P*Hi*128), box (64, 128)
                      const IdxPrefillArgs a) {
   extern __shared__ __align__(1024) uint8_t dsmem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
@@ -146,6 +146,7 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
     }
     uint32_t kit = 0, uit = 0;
     uint32_t used = 0, parity_bits = 0;   // key ring slots: issued at least once / parity of the last issue
+    const uint64_t pol_k = l2_policy_evict_last();   // a group's keys are read by every query tile
     int q_parity0 = -1, q_parity1 = -1;
     IdxUnit u;
     for (int k = 0; get_unit(k, u) && !s_abort; ++k) {
@@ -186,8 +187,9 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
             if (ok) {
               uint8_t* dst = k_smem + st * IDXP_STAGE_BYTES;
               mbar_arrive_expect_tx(&k_full[st], IDXP_STAGE_BYTES);
-              tma_load_4d(dst, &tmap_k, &k_full[st], 0, 0, u.g * a.hg + hl, page0);
-              tma_load_4d(dst + head_bytes, &tmap_k, &k_full[st], 0, 0, u.g * a.hg + hl, page1);
+              const int h = u.g * a.hg + hl;    // key rows of (page, head): one contiguous 16 KiB box
+              tma_load_2d_hint(dst, &tmap_k, &k_full[st], 0, (page0 * a.Hi + h) * 128, pol_k);
+              tma_load_2d_hint(dst + head_bytes, &tmap_k, &k_full[st], 0, (page1 * a.Hi + h) * 128, pol_k);
               used |= 1u << st;
               parity_bits = (parity_bits & ~(1u << st)) | (((kit / a.stages) & 1u) << st);
             }

@@ -221,10 +221,10 @@ msa_status_t launch_index_prefill(const msa_config_t* cfg, const msa_batch_t* ba
             msa::IDXP_MAXSEQ);
   CUtensorMap tk;
   {
-    const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
-    const uint64_t strides[3] = {128, 128 * 128, static_cast<uint64_t>(Hi) * 128 * 128};
-    const uint32_t box[4] = {64, 128, 1, 1};
-    if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box)) != MSA_OK) return st;
+    const uint64_t dims[2] = {64, static_cast<uint64_t>(batch->num_pages) * Hi * 128};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {64, 128};
+    if ((st = make_map(&tk, idx_k_cache, 2, dims, strides, box)) != MSA_OK) return st;
   }
   CUtensorMap tq;
   {
