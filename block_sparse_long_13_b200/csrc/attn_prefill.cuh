@@ -31,8 +31,8 @@ namespace msa {
 
 constexpr int ATTP_THREADS = 384;  // warpgroup 0: producer + UMMA warps; warpgroups 1, 2: softmax
 // Register split (setmaxnreg): the launch gives 168 per thread (65536 / 384, rounded to 8); warpgroup 0
-// returns registers, the softmax warpgroups take them.  128*56 + 256*224 = 64512 = 384*168.
-constexpr int ATTP_REGS_CTRL = 56, ATTP_REGS_SOFTMAX = 224;
+// returns registers, the softmax warpgroups take them.  128*72 + 256*216 = 64512 = 384*168.
+constexpr int ATTP_REGS_CTRL = 72, ATTP_REGS_SOFTMAX = 216;
 static_assert(128 * ATTP_REGS_CTRL + 256 * ATTP_REGS_SOFTMAX <= 384 * 168, "register split exceeds the launch");
 constexpr int ATTP_TOK = 8;       // tokens per tile (x 16 heads = 128 MMA rows)
 constexpr int ATTP_G = 16;        // query heads per KV group
@@ -350,9 +350,15 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
     // Tile i: S(i) = Q K^T into S[i % 2] (A and B from shared memory), then O = P(i-1) V with
     // P(i-1) read from TMEM.  tcgen05.commit tracks every earlier MMA of this thread, so the
     // s_full(i) signal also means PV(i-2) has finished reading P[i % 2].
+    // This one thread's instruction latency is on the critical path: descriptors are built once
+    // (only the 14-bit start address, in 16-byte units, moves) and ring positions are counters.
     const uint32_t id_s = idesc_bf16(128, 128, false, false);
     const uint32_t id_pv = idesc_bf16(128, 128, false, true);
-    const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s);
+    const uint64_t qdesc0 = sdesc_sw128(smem_u32(q_s), 16, 1024);
+    const uint64_t kdesc0 = sdesc_sw128(smem_u32(k_s), 16, 1024);
+    const uint64_t vdesc0 = sdesc_sw128(smem_u32(v_s), 16384, 1024);
+    int qb = 0;
+    uint32_t qph = 0;
     int cur_bucket = -1;
     uint32_t kvit = 0;
     bool pv_pending = false;
@@ -362,10 +368,8 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
       if (!mbar_wait(&o_empty, (j & 1) ^ 1, &s_abort)) return false;   // tile j-1's O has been read
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t bdesc = sdesc_sw128(va + kk * 2048, 16384, 1024);
-        umma_bf16_ts(tmem + ATTP_TM_O, tmem + ATTP_TM_P + pb * 64 + kk * 8, bdesc, id_pv, kk > 0 ? 1u : 0u);
-      }
+      for (int kk = 0; kk < 8; ++kk)   // 16 keys per step: 2048 bytes of V rows
+        umma_bf16_ts(tmem + ATTP_TM_O, tmem + ATTP_TM_P + pb * 64 + kk * 8, vdesc0 + 128 * kk, id_pv, kk > 0 ? 1u : 0u);
       umma_commit(&o_full[pb]);
       return true;
     };
@@ -384,18 +388,19 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
         ++kvit;
         cur_bucket = bucket;
       }
-      const int qb = i % ATTP_QBUF, sb = i & 1;
-      if (!mbar_wait(&q_full[qb], (i / ATTP_QBUF) & 1, &s_abort)) break;
+      const int sb = i & 1;
+      if (!mbar_wait(&q_full[qb], qph, &s_abort)) break;
       tc_fence_after();
       const uint32_t d = tmem + ATTP_TM_S + sb * 128;
+      const uint64_t qd = qdesc0 + static_cast<uint64_t>((qb * ATTP_QBYTES) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        umma_bf16_ss(d, sdesc_sw128(qa + qb * ATTP_QBYTES + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), id_s,
-                     kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < 8; ++kk) {   // 16 dims per step: 32 bytes within a 128-byte row, halves 16 KiB apart
+        const uint32_t off16 = (kk >> 2) * 1024 + (kk & 3) * 2;
+        umma_bf16_ss(d, qd + off16, kdesc0 + off16, id_s, kk > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[sb]);
       umma_commit(&q_empty[qb]);
+      if (++qb == ATTP_QBUF) { qb = 0; qph ^= 1u; }
       if (pv_pending) ok = issue_pv(i - 1);
       pv_pending = true;
     }

@@ -28,7 +28,7 @@ namespace msa {
 constexpr int IDXP_THREADS = 384;   // warpgroup 0: producer + UMMA warps; warpgroups 1, 2: epilogue
 // Register split (setmaxnreg; registers are granted per warpgroup): the launch gives 168 per thread
 // (65536 / 384, rounded to 8); warpgroup 0 returns registers, the epilogue warpgroups take them.
-constexpr int IDXP_REGS_CTRL = 64, IDXP_REGS_EPI = 216;
+constexpr int IDXP_REGS_CTRL = 72, IDXP_REGS_EPI = 216;
 static_assert(128 * IDXP_REGS_CTRL + 256 * IDXP_REGS_EPI <= 384 * 168, "register split exceeds the launch");
 constexpr int IDXP_TILE = 128;
 constexpr int IDXP_MAXSEQ = 1024;
@@ -207,33 +207,40 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ UMMA issuer
+    // One thread issues everything, so its own instruction latency is on the critical path: the
+    // descriptors are built once (only the 14-bit start address, in 16-byte units, moves between
+    // MMAs) and the ring positions are counters, not divisions.
     const uint32_t idesc = idesc_bf16(128, 256, false, false);
-    const uint32_t q_addr = smem_u32(q_smem), k_addr = smem_u32(k_smem);
-    uint32_t kit = 0, uit = 0, ait = 0;
+    const uint64_t qdesc0 = sdesc_sw128(smem_u32(q_smem), 16, 1024);
+    const uint64_t kdesc0 = sdesc_sw128(smem_u32(k_smem), 16, 1024);
+    int st = 0, buf = 0;                    // key stage, accumulator buffer
+    uint32_t kph = 0, aph = 0;              // phase of the key ring's current lap; accumulator use count / 2
+    uint32_t uit = 0;
     IdxUnit u;
     for (int k = 0; get_unit(k, u) && !s_abort; ++k) {
       if (u.nblk == 0) continue;
-      const int qb = uit % a.nqbuf;
-      if (!mbar_wait(&q_full[qb], (uit / a.nqbuf) & 1, &s_abort)) break;
+      const int qb = a.nqbuf == 1 ? 0 : static_cast<int>(uit & 1);
+      const uint32_t qpar = a.nqbuf == 1 ? (uit & 1) : ((uit >> 1) & 1);
+      if (!mbar_wait(&q_full[qb], qpar, &s_abort)) break;
       ++uit;
-      const int nstep = ((u.nblk + 1) >> 1) * a.hg;
+      const int npair = (u.nblk + 1) >> 1;
       bool ok = true;
-      for (int sp = 0; sp < nstep; ++sp, ++kit, ++ait) {
-        const int hl = sp % a.hg;
-        const int st = kit % a.stages;
-        const int buf = ait & 1;
-        if (!mbar_wait(&acc_empty[buf], ((ait >> 1) & 1) ^ 1, &s_abort)) { ok = false; break; }
-        if (!mbar_wait(&k_full[st], (kit / a.stages) & 1, &s_abort)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d = tmem + static_cast<uint32_t>(buf * 256);
-        const uint32_t qa = q_addr + qb * q_bytes + hl * head_bytes;
-        const uint32_t ka = k_addr + st * IDXP_STAGE_BYTES;   // 256 key rows: two blocks
+      for (int pr = 0; pr < npair && ok; ++pr) {
+        for (int hl = 0; hl < a.hg; ++hl) {
+          if (!mbar_wait(&acc_empty[buf], (aph & 1) ^ 1, &s_abort)) { ok = false; break; }
+          if (!mbar_wait(&k_full[st], kph, &s_abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + static_cast<uint32_t>(buf * 256);
+          const uint64_t qd = qdesc0 + static_cast<uint64_t>((qb * q_bytes + hl * head_bytes) >> 4);
+          const uint64_t kd = kdesc0 + static_cast<uint64_t>((st * IDXP_STAGE_BYTES) >> 4);   // two blocks
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16_ss(d, sdesc_sw128(qa + kk * 32, 16, 1024), sdesc_sw128(ka + kk * 32, 16, 1024), idesc,
-                       kk > 0 ? 1u : 0u);
-        umma_commit(&k_empty[st]);
-        umma_commit(&acc_full[buf]);
+          for (int kk = 0; kk < 4; ++kk) umma_bf16_ss(d, qd + 2 * kk, kd + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+          umma_commit(&k_empty[st]);
+          umma_commit(&acc_full[buf]);
+          if (++st == a.stages) { st = 0; kph ^= 1u; }
+          aph += buf;                          // one full use of both buffers per two steps
+          buf ^= 1;
+        }
       }
       umma_commit(&q_empty[qb]);  // the query tile is free once this unit's MMAs are done
       if (!ok) break;
