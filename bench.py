@@ -436,7 +436,7 @@ def main():
                 addk("index_prefill_kernel (fused top-k)", c["index_ms"], 1, flops=c["index"]["flops"])
             else:
                 addk("index_prefill_kernel", c["index_ms"], 1, flops=c["index"]["flops"])
-                addk("topk_blocks_kernel (prefill)", c["topk_ms"], 1, bytes_=c["topk"]["bytes"])
+                addk("topk kernel (prefill)", c["topk_ms"], 1, bytes_=c["topk"]["bytes"])
             ph = c["attn_phases"]
             if ph is not None:
                 addk("schedule (4 kernels)", ph["schedule_ms"], 4)
@@ -444,7 +444,7 @@ def main():
                 addk("attn_merge_kernel", ph["merge_ms"], 1, bytes_=c["merge"]["bytes"])
         else:
             addk("index_decode_kernel", c["index_ms"], 1, bytes_=c["index"]["bytes"])
-            addk("topk_blocks_kernel (decode)", c["topk_ms"], 1, bytes_=c["topk"]["bytes"])
+            addk("topk kernel (decode)", c["topk_ms"], 1, bytes_=c["topk"]["bytes"])
             addk("attn_decode_kernel", c["attn_ms"], 1, bytes_=c["attn"]["bytes"])
     # every kernel is timed inside a step of tens of ms: the sustained tensor peak is the denominator
     tensor_peak, tensor_src = pk["bf16_tflops_sustained"], pk["source"] + " sustained bf16 (cuBLAS, power-capped)"
