@@ -223,24 +223,35 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
       const uint32_t qpar = a.nqbuf == 1 ? (uit & 1) : ((uit >> 1) & 1);
       if (!mbar_wait(&q_full[qb], qpar, &s_abort)) break;
       ++uit;
-      const int npair = (u.nblk + 1) >> 1;
-      bool ok = true;
-      for (int pr = 0; pr < npair && ok; ++pr) {
-        for (int hl = 0; hl < a.hg; ++hl) {
-          if (!mbar_wait(&acc_empty[buf], (aph & 1) ^ 1, &s_abort)) { ok = false; break; }
-          if (!mbar_wait(&k_full[st], kph, &s_abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem + static_cast<uint32_t>(buf * 256);
-          const uint64_t qd = qdesc0 + static_cast<uint64_t>((qb * q_bytes + hl * head_bytes) >> 4);
-          const uint64_t kd = kdesc0 + static_cast<uint64_t>((st * IDXP_STAGE_BYTES) >> 4);   // two blocks
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) umma_bf16_ss(d, qd + 2 * kk, kd + 2 * kk, idesc, kk > 0 ? 1u : 0u);
-          umma_commit(&k_empty[st]);
-          umma_commit(&acc_full[buf]);
-          if (++st == a.stages) { st = 0; kph ^= 1u; }
-          aph += buf;                          // one full use of both buffers per two steps
-          buf ^= 1;
-        }
+      // The tensor pipe queues about one MMA: the barriers of step sp + 1 are awaited while the first
+      // two MMAs of step sp run, so the next step's MMAs are ready when the pipe frees up.
+      const int nstep = ((u.nblk + 1) >> 1) * a.hg;
+      bool ok = nstep > 0 && mbar_wait(&acc_empty[buf], (aph & 1) ^ 1, &s_abort) && mbar_wait(&k_full[st], kph, &s_abort);
+      int hl = 0;
+      for (int sp = 0; sp < nstep && ok; ++sp) {
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(buf * 256);
+        const uint64_t qd = qdesc0 + static_cast<uint64_t>((qb * q_bytes + hl * head_bytes) >> 4);
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>((st * IDXP_STAGE_BYTES) >> 4);   // two blocks
+        umma_bf16_ss(d, qd, kd, idesc, 0u);
+        umma_bf16_ss(d, qd + 2, kd + 2, idesc, 1u);
+        // positions of the next step, and its barriers
+        int st2 = st + 1;
+        uint32_t kph2 = kph;
+        if (st2 == a.stages) { st2 = 0; kph2 ^= 1u; }
+        const int buf2 = buf ^ 1;
+        const uint32_t aph2 = aph + static_cast<uint32_t>(buf);
+        if (sp + 1 < nstep)
+          ok = mbar_wait(&acc_empty[buf2], (aph2 & 1) ^ 1, &s_abort) && mbar_wait(&k_full[st2], kph2, &s_abort);
+        umma_bf16_ss(d, qd + 4, kd + 4, idesc, 1u);
+        umma_bf16_ss(d, qd + 6, kd + 6, idesc, 1u);
+        umma_commit(&k_empty[st]);
+        umma_commit(&acc_full[buf]);
+        st = st2;
+        kph = kph2;
+        buf = buf2;
+        aph = aph2;
+        if (++hl == a.hg) hl = 0;
       }
       umma_commit(&q_empty[qb]);  // the query tile is free once this unit's MMAs are done
       if (!ok) break;
