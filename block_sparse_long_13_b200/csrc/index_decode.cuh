@@ -14,22 +14,27 @@
 // page) units.  Warp 0 is the producer: it reads the page ids of 32 units at
 // a time (one coalesced load) and streams each unit as H_kv TMA tiles of
 // hg x 128 x 64 bf16 (128-byte swizzle) through a ring of shared buffers
-// guarded by full/empty mbarriers.  Warps 1..8 consume: each thread owns one
-// key row, widens it to fp32 and dots it with the sequence's (<= 8) queries
-// held in shared memory; the block max is a warp redux.sync on
-// order-preserving integer keys, then a per-group sum over the heads.
+// guarded by full/empty mbarriers.  The consumers are groups of 8 warps; a
+// group takes every NG-th stage (NG = 2 for at most 2 queries per sequence,
+// so one group's per-stage barrier and reduction latency hides behind the
+// other's work; else 1).  In a group each thread owns one key row, widens it
+// to fp32 and dots it with the sequence's (<= 8) queries held in shared
+// memory; the block max is a warp redux.sync on order-preserving integer
+// keys, then a per-group sum over the heads.
 #pragma once
 #include "common.cuh"
 
 namespace msa {
 
-constexpr int IDXD_CONSUMERS = 256;
-constexpr int IDXD_THREADS = 32 + IDXD_CONSUMERS;
+constexpr int IDXD_CONSUMERS = 256;   // threads of one consumer group
+// consumer groups for a query bound NQ (the register budget of two groups fits NQ <= 2)
+__host__ __device__ constexpr int idxd_groups(int nq) { return nq <= 2 ? 2 : 1; }
+__host__ __device__ constexpr int idxd_threads(int nq) { return 32 + IDXD_CONSUMERS * idxd_groups(nq); }
 constexpr int IDXD_MAXQ = 8;       // queries per sequence handled by this form
 constexpr int IDXD_MAXHG = 8;      // indexer heads per KV group
 constexpr int IDXD_MAXHI = 16;     // indexer heads
 constexpr int IDXD_MAXSEQ = 2048;  // sequences per call for this form
-constexpr int IDXD_SMEM_BUDGET = 212 * 1024;  // dynamic: key ring + this call's queries
+constexpr int IDXD_SMEM_BUDGET = 212 * 1024;  // dynamic: key ring + each group's queries
 
 struct IdxDecodeArgs {
   const __nv_bfloat16* idx_q;   // [total_q][Hi][64]
@@ -43,15 +48,16 @@ struct IdxDecodeArgs {
 
 // NQ: compile-time bound on the queries of any sequence (1, 2, 4 or 8)
 template <int NQ>
-__global__ void __launch_bounds__(IDXD_THREADS, 1)
+__global__ void __launch_bounds__(idxd_threads(NQ), 1)
 index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeArgs a) {
+  constexpr int NG = idxd_groups(NQ);
   extern __shared__ __align__(1024) uint8_t dsmem[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t full_bar[16], empty_bar[16];
   __shared__ int s_nbprefix[IDXD_MAXSEQ + 1];
-  __shared__ uint32_t s_part[2][NQ][IDXD_MAXHG][4];
-  // current sequence's queries of all heads, fp32, after the key ring
-  float* s_q = reinterpret_cast<float*>(ring + static_cast<long>(a.stages) * a.stage_bytes);
+  __shared__ uint32_t s_part[NG][2][NQ][IDXD_MAXHG][4];
+  // per consumer group: its current sequence's queries of all heads, fp32, after the key ring
+  float* s_q_all = reinterpret_cast<float*>(ring + static_cast<long>(a.stages) * a.stage_bytes);
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x;
@@ -135,51 +141,57 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
   } else {
     // ------------------------------------------------------------ consumers
     const int c = tid - 32;
-    const int cw = c >> 5;               // consumer warp 0..7
-    const int token = c & 127;
-    const int hl0 = c >> 7;              // 0 or 1
+    const int grp = c / IDXD_CONSUMERS;   // group: stages k = grp, grp + NG, ...
+    const int cl = c % IDXD_CONSUMERS;
+    const int cw = cl >> 5;               // warp of the group, 0..7
+    const int token = cl & 127;
+    const int hl0 = cl >> 7;              // 0 or 1
+    const int bar_seq = 1 + 2 * grp, bar_stage = 2 + 2 * grp;   // the group's named barriers
+    float* s_q = s_q_all + grp * (NQ * a.Hi * 64);
     int cur_seq = -1, nq = 0, qrow0 = 0, ctx = 0;
     int s, b;
     locate(u0, s, b);
-    // the per-group sum of stage k-1 is made after the barrier that opens stage k
+    long cur_unit = 0;                    // unit (s, b) stands for, within this CTA
+    // the per-group sum of the group's previous stage is made after the barrier that opens the next one
     int pv_nq = 0, pv_row0 = 0, pv_g = 0, pv_b = 0;
     auto combine = [&](int pbuf) {
-      if (c < pv_nq) {
+      if (cl < pv_nq) {
         float tot = 0.f;
         for (int hl = 0; hl < a.hg; ++hl) {
-          const uint32_t* pp = s_part[pbuf][c][hl];
+          const uint32_t* pp = s_part[grp][pbuf][cl][hl];
           tot += key_to_float(max(max(pp[0], pp[1]), max(pp[2], pp[3])));
         }
-        a.scores[(static_cast<long>(pv_row0 + c) * a.Hkv + pv_g) * a.max_blocks + pv_b] = tot;
+        a.scores[(static_cast<long>(pv_row0 + cl) * a.Hkv + pv_g) * a.max_blocks + pv_b] = tot;
       }
     };
     bool ok = true;
-    for (long k = 0; k < nstage; ++k) {
+    int m = 0;                            // stages taken by this group so far
+    for (long k = grp; k < nstage; k += NG, ++m) {
       const int g = static_cast<int>(k % a.Hkv);
-      if (k > 0 && g == 0) {  // next unit: next block, or the next sequence with blocks
+      for (const long unit = k / a.Hkv; cur_unit < unit; ++cur_unit) {   // next block, or next sequence with blocks
         ++b;
         while (b >= s_nbprefix[s + 1] - s_nbprefix[s]) { ++s; b = 0; }
       }
       if (s != cur_seq) {
         // this sequence's queries (all indexer heads) as fp32
-        named_bar_sync(1, IDXD_CONSUMERS);
+        named_bar_sync(bar_seq, IDXD_CONSUMERS);
         cur_seq = s;
         qrow0 = __ldg(a.q_start + s);
         nq = __ldg(a.q_start + s + 1) - qrow0;
         ctx = __ldg(a.ctx_len + s);
-        if (nq > NQ) { if (c == 0) flag_error(MSA_DEV_BOUNDS); nq = NQ; }
+        if (nq > NQ) { if (cl == 0) flag_error(MSA_DEV_BOUNDS); nq = NQ; }
         const int n = nq * a.Hi * 64;
         const __nv_bfloat16* src = a.idx_q + static_cast<long>(qrow0) * a.Hi * 64;
-        for (int i = c; i < n; i += IDXD_CONSUMERS) s_q[i] = __bfloat162float(src[i]);
-        named_bar_sync(1, IDXD_CONSUMERS);
+        for (int i = cl; i < n; i += IDXD_CONSUMERS) s_q[i] = __bfloat162float(src[i]);
+        named_bar_sync(bar_seq, IDXD_CONSUMERS);
       }
       const int slot = static_cast<int>(k % a.stages);
       const uint32_t par = static_cast<uint32_t>((k / a.stages) & 1);
-      if (!mbar_wait_group(&full_bar[slot], par, &s_abort, 2, IDXD_CONSUMERS)) { ok = false; break; }
-      if (k > 0) combine(static_cast<int>((k - 1) & 1));
+      if (!mbar_wait_group(&full_bar[slot], par, &s_abort, bar_stage, IDXD_CONSUMERS)) { ok = false; break; }
+      if (m > 0) combine((m - 1) & 1);
       const uint8_t* tile = ring + static_cast<long>(slot) * a.stage_bytes;
       const int j = b * a.block_size + token;  // absolute key position
-      const int pbuf = static_cast<int>(k & 1);
+      const int pbuf = m & 1;
       for (int hl = hl0; hl < a.hg; hl += 2) {
         // this thread's key row: 64 bf16, 128-byte swizzled
         const uint8_t* rowp = tile + (hl * 128 + token) * 128;
@@ -209,8 +221,8 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
           if (NQ == 1 || i < nq) {
             const int p = ctx - nq + i;
             const float v = (j <= p) ? ac0[i] + ac1[i] : -INFINITY;
-            const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, order_key(v));
-            if (lane == 0) s_part[pbuf][i][hl][cw & 3] = m;
+            const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, order_key(v));
+            if (lane == 0) s_part[grp][pbuf][i][hl][cw & 3] = mx;
           }
         }
       }
@@ -218,9 +230,9 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
       if (lane == 0) mbar_arrive(&empty_bar[slot]);  // this warp is done with the tile
       pv_nq = nq; pv_row0 = qrow0; pv_g = g; pv_b = b;
     }
-    if (ok && nstage > 0) {
-      named_bar_sync(1, IDXD_CONSUMERS);               // last stage's partial maxima visible
-      combine(static_cast<int>((nstage - 1) & 1));
+    if (ok && m > 0) {
+      named_bar_sync(bar_seq, IDXD_CONSUMERS);          // the group's last partial maxima visible
+      combine((m - 1) & 1);
     }
   }
 }
