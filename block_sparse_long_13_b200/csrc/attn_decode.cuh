@@ -10,10 +10,11 @@
 // restriction is the "Indexer-selected sparse attention" row.
 //
 // One CTA per (row, group, split); a split owns a contiguous run of the
-// row's selected slots.  Inside a CTA, thread i owns key i of the current
-// 128-token block for Q.K (16 head dot products of length 128), then thread d
-// owns output dimension d for P.V; running max / sum per head follow the
-// usual online-softmax recurrence in the log2 domain.  Splits of a unit write
+// row's selected slots.  Per selected block, one bulk copy brings V_b (32 KiB)
+// into shared memory while thread i loads key row i (all 16 pieces in flight)
+// and makes its 16 head dot products; for P.V thread (dp, hh) owns output
+// dimensions 2dp, 2dp+1 of heads 8hh..8hh+7.  Running max / sum per head
+// follow the usual online-softmax recurrence in the log2 domain.  Splits of a unit write
 // (O, lse) partials to the workspace; the last split to finish (device
 // counter) merges them by log-sum-exp ("LSE fusion", "Two-phase forward").
 #pragma once
@@ -24,6 +25,8 @@ namespace msa {
 constexpr int ATTD_THREADS = 128;
 constexpr int ATTD_G = 16;     // query heads per KV group handled by this kernel
 constexpr int ATTD_D = 128;    // head_dim
+constexpr int ATTD_VBYTES = 128 * ATTD_D * 2;          // one V block, bf16
+constexpr int ATTD_SMEM = ATTD_VBYTES + 128;           // dynamic: V block (+ alignment)
 
 struct AttnDecodeArgs {
   const __nv_bfloat16* q;        // [total_q][Hq][128]
@@ -50,13 +53,18 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __global__ void __launch_bounds__(ATTD_THREADS)
 attn_decode_kernel(const AttnDecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __nv_bfloat16* s_v = reinterpret_cast<__nv_bfloat16*>((reinterpret_cast<uintptr_t>(dsm) + 127) & ~uintptr_t(127));
   __shared__ __align__(16) float s_q[ATTD_G * ATTD_D];     // scaled queries (log2 domain)
   __shared__ __align__(16) float s_p[ATTD_G * 128];        // probabilities of the current block
   __shared__ float s_red[4][ATTD_G];
   __shared__ float s_m[ATTD_G], s_l[ATTD_G], s_alpha[ATTD_G];
   __shared__ int s_last;
+  __shared__ uint64_t v_full;
+  __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int dp = tid & 63, hh = tid >> 6;            // P.V: dims 2dp, 2dp+1 of heads 8hh .. 8hh+7
   const long unit = blockIdx.x / a.nsplit;           // (t, g)
   const int split = blockIdx.x % a.nsplit;
   const int t = static_cast<int>(unit / a.Hkv);
@@ -66,18 +74,25 @@ attn_decode_kernel(const AttnDecodeArgs a) {
   const int nq = __ldg(a.q_start + s + 1) - qs;
   const int p = __ldg(a.ctx_len + s) - nq + (t - qs);
 
+  if (tid == 0) {
+    s_abort = 0;
+    mbar_init(&v_full, 1);
+    fence_mbar_init();
+  }
   // queries of the group, pre-scaled into the log2 domain
   const __nv_bfloat16* qg = a.q + (static_cast<long>(t) * a.Hq + g * ATTD_G) * ATTD_D;
   for (int i = tid; i < ATTD_G * ATTD_D; i += ATTD_THREADS) s_q[i] = __bfloat162float(qg[i]) * a.scale_log2;
   if (tid < ATTD_G) { s_m[tid] = -INFINITY; s_l[tid] = 0.f; }
-  float o_acc[ATTD_G];
+  float o_acc[8][2];
 #pragma unroll
-  for (int h = 0; h < ATTD_G; ++h) o_acc[h] = 0.f;
+  for (int k = 0; k < 8; ++k) { o_acc[k][0] = 0.f; o_acc[k][1] = 0.f; }
   __syncthreads();
 
   const int per = (a.topk + a.nsplit - 1) / a.nsplit;
   const int slot0 = split * per, slot1 = min(a.topk, slot0 + per);
   const int32_t* sel = a.block_idx + unit * a.topk;
+  uint32_t vph = 0;                                  // V copies issued so far (parity of the next wait)
+  bool v_pending = false;
   for (int slot = slot0; slot < slot1; ++slot) {
     const int b = __ldg(sel + slot);
     if (b < 0) continue;  // uniform across the CTA
@@ -85,16 +100,25 @@ attn_decode_kernel(const AttnDecodeArgs a) {
     int page = __ldg(a.page_table + static_cast<long>(s) * a.max_blocks + b);
     if (page < 0 || page >= a.num_pages) { if (tid == 0) flag_error(MSA_DEV_BOUNDS); continue; }
     const long base = (static_cast<long>(page) * a.Hkv + g) * 128 * ATTD_D;
+    // V_b into shared memory (the previous block's readers are past the barrier that ended its loop)
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&v_full, ATTD_VBYTES);
+      bulk_load(s_v, a.v_cache + base, ATTD_VBYTES, &v_full);
+    }
+    v_pending = true;
 
-    // --- S = q K^T for key tid (16 heads)
+    // --- S = q K^T for key tid (16 heads); the row's 16 pieces are loaded before use
     const int j = b * a.block_size + tid;
     const uint4* krow = reinterpret_cast<const uint4*>(a.k_cache + base + static_cast<long>(tid) * ATTD_D);
+    uint4 kw[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) kw[c] = __ldg(krow + c);
     float sc[ATTD_G];
 #pragma unroll
     for (int h = 0; h < ATTD_G; ++h) sc[h] = 0.f;
-#pragma unroll 4
+#pragma unroll
     for (int c = 0; c < 16; ++c) {
-      const uint4 w = __ldg(krow + c);
+      const uint4 w = kw[c];
       const float kf[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
                            bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
 #pragma unroll
@@ -131,25 +155,53 @@ attn_decode_kernel(const AttnDecodeArgs a) {
       const float ws = warp_sum(pv);
       if (lane == 0) s_red[warp][h] = ws;
     }
-    __syncthreads();
+    const bool v_ok = mbar_wait(&v_full, vph & 1, &s_abort);
+    ++vph;
+    v_pending = !v_ok;
+    if (__syncthreads_or(!v_ok)) break;       // s_p, s_red and V_b visible to every thread
     if (tid < ATTD_G) s_l[tid] = s_l[tid] * s_alpha[tid] + (s_red[0][tid] + s_red[1][tid]) + (s_red[2][tid] + s_red[3][tid]);
-    // --- O = alpha O + P V for output dim tid
+    // --- O = alpha O + P V, keys in groups of 4 (P as float4), keys past the row's position skipped
 #pragma unroll
-    for (int h = 0; h < ATTD_G; ++h) o_acc[h] *= s_alpha[h];
-    const __nv_bfloat16* vcol = a.v_cache + base + tid;
+    for (int k = 0; k < 8; ++k) {
+      const float al = s_alpha[8 * hh + k];
+      o_acc[k][0] *= al;
+      o_acc[k][1] *= al;
+    }
+    const uint32_t* vcol = reinterpret_cast<const uint32_t*>(s_v) + dp;   // V[i][2dp .. 2dp+1] at vcol[64 i]
+    const float* prow = s_p + (8 * hh) * 128;
     const int nvis = min(128, p - b * a.block_size + 1);
-#pragma unroll 4
-    for (int i = 0; i < nvis; ++i) {
-      const float v = __bfloat162float(vcol[static_cast<long>(i) * ATTD_D]);
+    int i0 = 0;
+    for (; i0 + 4 <= nvis; i0 += 4) {
+      float4 pw[8];
 #pragma unroll
-      for (int h4 = 0; h4 < ATTD_G; h4 += 4) {
-        o_acc[h4 + 0] = fmaf(s_p[(h4 + 0) * 128 + i], v, o_acc[h4 + 0]);
-        o_acc[h4 + 1] = fmaf(s_p[(h4 + 1) * 128 + i], v, o_acc[h4 + 1]);
-        o_acc[h4 + 2] = fmaf(s_p[(h4 + 2) * 128 + i], v, o_acc[h4 + 2]);
-        o_acc[h4 + 3] = fmaf(s_p[(h4 + 3) * 128 + i], v, o_acc[h4 + 3]);
+      for (int k = 0; k < 8; ++k) pw[k] = *reinterpret_cast<const float4*>(prow + k * 128 + i0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t vv = vcol[(i0 + u) * 64];
+        const float v0 = bf16lo(vv), v1 = bf16hi(vv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float pk = u == 0 ? pw[k].x : u == 1 ? pw[k].y : u == 2 ? pw[k].z : pw[k].w;
+          o_acc[k][0] = fmaf(pk, v0, o_acc[k][0]);
+          o_acc[k][1] = fmaf(pk, v1, o_acc[k][1]);
+        }
       }
     }
-    __syncthreads();  // s_p / s_l / s_alpha reused by the next block
+    for (; i0 < nvis; ++i0) {
+      const uint32_t vv = vcol[i0 * 64];
+      const float v0 = bf16lo(vv), v1 = bf16hi(vv);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float pk = prow[k * 128 + i0];
+        o_acc[k][0] = fmaf(pk, v0, o_acc[k][0]);
+        o_acc[k][1] = fmaf(pk, v1, o_acc[k][1]);
+      }
+    }
+    __syncthreads();  // s_p / s_l / s_alpha / V_b reused by the next block
+  }
+  if (s_abort) {                                     // a V copy that did not land in time: let it finish
+    if (tid == 0 && v_pending) mbar_wait_drain(&v_full, (vph - 1) & 1);
+    return;
   }
 
   // ---- finish: this split's (O / l, lse)
@@ -157,9 +209,12 @@ attn_decode_kernel(const AttnDecodeArgs a) {
   if (a.nsplit == 1) {
     __nv_bfloat16* orow = a.out + (static_cast<long>(t) * a.Hq + g * ATTD_G) * ATTD_D;
 #pragma unroll
-    for (int h = 0; h < ATTD_G; ++h) {
+    for (int k = 0; k < 8; ++k) {
+      const int h = 8 * hh + k;
       const float l = s_l[h];
-      orow[h * ATTD_D + tid] = __float2bfloat16_rn(l > 0.f ? o_acc[h] / l : 0.f);
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      *reinterpret_cast<__nv_bfloat162*>(orow + h * ATTD_D + 2 * dp) =
+          __floats2bfloat162_rn(o_acc[k][0] * inv, o_acc[k][1] * inv);
     }
     if (a.lse && tid < ATTD_G) {
       const float l = s_l[tid];
@@ -169,9 +224,11 @@ attn_decode_kernel(const AttnDecodeArgs a) {
   }
   float* po = a.part_o + (unit * a.nsplit + split) * (ATTD_G * ATTD_D);
 #pragma unroll
-  for (int h = 0; h < ATTD_G; ++h) {
+  for (int k = 0; k < 8; ++k) {
+    const int h = 8 * hh + k;
     const float l = s_l[h];
-    po[h * ATTD_D + tid] = l > 0.f ? o_acc[h] / l : 0.f;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    *reinterpret_cast<float2*>(po + h * ATTD_D + 2 * dp) = make_float2(o_acc[k][0] * inv, o_acc[k][1] * inv);
   }
   if (tid < ATTD_G) {
     const float l = s_l[tid];

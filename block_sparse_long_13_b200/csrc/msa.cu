@@ -526,7 +526,8 @@ msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, 
   a.scale_log2 = softmax_scale(cfg) * 1.4426950408889634f;
   const size_t units = static_cast<size_t>(batch->total_q) * cfg->num_kv_heads;
   CUDA_TRY(cudaMemsetAsync(a.counters, 0, units * 4, stream));
-  msa::attn_decode_kernel<<<static_cast<unsigned>(units * w.nsplit), msa::ATTD_THREADS, 0, stream>>>(a);
+  CUDA_TRY(set_smem(msa::attn_decode_kernel, msa::ATTD_SMEM));   // with the static arrays: above the 48 KiB default
+  msa::attn_decode_kernel<<<static_cast<unsigned>(units * w.nsplit), msa::ATTD_THREADS, msa::ATTD_SMEM, stream>>>(a);
   return launched();
 }
 
