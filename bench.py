@@ -505,24 +505,56 @@ def main():
             h2d += sum(t.numel() * t.element_size() for t in new_kv.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out)
 
+        # Copies in run on s_in, the calls on the compute stream, copies out on s_out, chained per part
+        # by events: part i's inputs arrive while part i-1 computes and its output leaves while part
+        # i+1 computes (a chunked prefill pipelines this way).  A device buffer is rewritten only after
+        # its previous use has finished: inputs after the previous step's call on them, outputs after
+        # the previous step's copy out, the prefill's caches after the previous step's last prefill call.
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        n = len(parts)
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_done = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        last_prefill = max((i for i, p in enumerate(parts) if p.kind == "prefill"), default=-1)
+        started = [False]
+
         def e2e_step():
-            if new_kv is not None:
-                for key, t in new_kv.items():
-                    parts[0].caches[key].copy_(t, non_blocking=True)
-            for p, hin in zip(parts, host_in):
-                p.q.copy_(hin["q"], non_blocking=True)
-                p.idx_q.copy_(hin["idx_q"], non_blocking=True)
-            step()
-            for p, hout in zip(parts, host_out):
-                hout.copy_(p.out, non_blocking=True)
+            again = started[0]
+            started[0] = True
+            with torch.cuda.stream(s_in):
+                if new_kv is not None:
+                    if again:
+                        s_in.wait_event(ev_done[last_prefill])
+                    for key, t in new_kv.items():
+                        parts[0].caches[key].copy_(t, non_blocking=True)
+                for i, (p, hin) in enumerate(zip(parts, host_in)):
+                    if again:
+                        s_in.wait_event(ev_done[i])
+                    p.q.copy_(hin["q"], non_blocking=True)
+                    p.idx_q.copy_(hin["idx_q"], non_blocking=True)
+                    ev_in[i].record(s_in)
+            for i, p in enumerate(parts):
+                stream.wait_event(ev_in[i])
+                if again:
+                    stream.wait_event(ev_out[i])
+                p.run(workspace, None, stream, args.stop_after)
+                ev_done[i].record(stream)
+            with torch.cuda.stream(s_out):
+                for i, (p, hout) in enumerate(zip(parts, host_out)):
+                    s_out.wait_event(ev_done[i])
+                    hout.copy_(p.out, non_blocking=True)
+                    ev_out[i].record(s_out)
         e2e_step()
+        stream.wait_stream(s_out)
         torch.cuda.synchronize()
         barrier(ws)
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
+        s_in.wait_event(a0)
         ksteps = max(2, args.steps // 2)
         for _ in range(ksteps):
             e2e_step()
+        stream.wait_stream(s_out)          # the timed region ends when the last output is on the host
         a1.record(stream)
         torch.cuda.synchronize()
         barrier(ws)
