@@ -509,24 +509,37 @@ def main():
         # by events: part i's inputs arrive while part i-1 computes and its output leaves while part
         # i+1 computes (a chunked prefill pipelines this way).  A device buffer is rewritten only after
         # its previous use has finished: inputs after the previous step's call on them, outputs after
-        # the previous step's copy out, the prefill's caches after the previous step's last prefill call.
+        # the previous step's copy out, each of the prefill's two alternating cache copies after the last
+        # prefill call that read it.
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
         n = len(parts)
         ev_in = [torch.cuda.Event() for _ in range(n)]
         ev_done = [torch.cuda.Event() for _ in range(n)]
         ev_out = [torch.cuda.Event() for _ in range(n)]
         last_prefill = max((i for i, p in enumerate(parts) if p.kind == "prefill"), default=-1)
-        started = [False]
+        # the prefill's own caches alternate between two device copies from step to step, so the next
+        # step's copy in does not wait for this step's last prefill call (a serving loop double-buffers
+        # its staging the same way)
+        cache_sets, cache_free = None, None
+        if new_kv is not None:
+            cache_sets = [parts[0].caches, {k: torch.empty_like(v) for k, v in parts[0].caches.items()}]
+            cache_free = [torch.cuda.Event(), torch.cuda.Event()]
+        started = [0]
 
         def e2e_step():
-            again = started[0]
-            started[0] = True
+            j = started[0]
+            again = j > 0
+            started[0] = j + 1
             with torch.cuda.stream(s_in):
                 if new_kv is not None:
-                    if again:
-                        s_in.wait_event(ev_done[last_prefill])
+                    cs = cache_sets[j % 2]
+                    if j >= 2:
+                        s_in.wait_event(cache_free[j % 2])      # its last reader, two steps back
                     for key, t in new_kv.items():
-                        parts[0].caches[key].copy_(t, non_blocking=True)
+                        cs[key].copy_(t, non_blocking=True)
+                    for p in parts:
+                        if p.kind == "prefill":
+                            p.caches = cs
                 for i, (p, hin) in enumerate(zip(parts, host_in)):
                     if again:
                         s_in.wait_event(ev_done[i])
@@ -539,6 +552,8 @@ def main():
                     stream.wait_event(ev_out[i])
                 p.run(workspace, None, stream, args.stop_after)
                 ev_done[i].record(stream)
+                if i == last_prefill and cache_free is not None:
+                    cache_free[j % 2].record(stream)
             with torch.cuda.stream(s_out):
                 for i, (p, hout) in enumerate(zip(parts, host_out)):
                     s_out.wait_event(ev_done[i])
@@ -556,6 +571,10 @@ def main():
             e2e_step()
         stream.wait_stream(s_out)          # the timed region ends when the last output is on the host
         a1.record(stream)
+        if cache_sets is not None:
+            for p in parts:
+                if p.kind == "prefill":
+                    p.caches = cache_sets[0]
         torch.cuda.synchronize()
         barrier(ws)
         ems = max_over_ranks(a0.elapsed_time(a1) / ksteps, ws)
