@@ -61,7 +61,7 @@ msa_status_t check_config(const msa_config_t* c) {
             "head counts and topk must be positive");
   CHECK_ARG(c->num_q_heads % c->num_kv_heads == 0, "num_q_heads must be a multiple of num_kv_heads");
   CHECK_ARG(c->idx_heads % c->num_kv_heads == 0, "idx_heads must be a multiple of num_kv_heads");
-  CHECK_SUP(c->num_q_heads / c->num_kv_heads == 16, "this build needs 16 query heads per KV head");
+  CHECK_SUP(c->num_q_heads / c->num_kv_heads == 16, "this library needs 16 query heads per KV head");
   CHECK_SUP(c->idx_heads / c->num_kv_heads <= 4, "at most 4 indexer heads per KV group");
   CHECK_SUP(c->idx_heads <= 16, "at most 16 indexer heads");
   CHECK_SUP(c->head_dim == 128, "head_dim must be 128");

@@ -69,7 +69,7 @@ extern "C" {
 typedef enum {
   MSA_OK = 0,
   MSA_ERR_INVALID_ARG = 1,  /* a pointer, size or layout argument is wrong        */
-  MSA_ERR_UNSUPPORTED = 2,  /* valid, but outside the sizes this build handles    */
+  MSA_ERR_UNSUPPORTED = 2,  /* valid, but outside the sizes this library handles  */
   MSA_ERR_CUDA = 3,         /* a CUDA runtime / driver call failed                 */
   MSA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (status query)   */
   MSA_ERR_DEVICE_BOUNDS = 5 /* the device found an out-of-range index (status)     */
