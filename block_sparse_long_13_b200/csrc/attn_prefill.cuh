@@ -60,32 +60,80 @@ __device__ __forceinline__ int entry_bucket(const SchedArgs& a, int t, int g, in
 }
 
 // pass = 0: count entries per bucket; pass = 1: scatter them.  Buckets are
-// many (sequences x groups x blocks) and each CTA's rows hit few entries of
-// each, so the counters are global atomics; the order of entries inside a
-// bucket is arbitrary and does not change any result.
+// many (sequences x groups x blocks), so the counters are global atomics; the
+// order of entries inside a bucket is arbitrary and does not change any result.
+// Blocks that most queries select (the planted or sink-like ones, each row's
+// own block) would take thousands of atomics on one address, so a CTA first
+// gathers its rows' entries per bucket in a shared-memory hash table and then
+// adds one count per distinct bucket; each entry's position is the bucket's
+// reserved base plus its rank inside the CTA.
+constexpr int SCHED_HASH = 4096;                  // table slots: >= 2 x a CTA's entries when it is used
+constexpr int SCHED_EPT = SCHED_HASH / 2 / 256;   // entries per thread (256 threads)
+
 __global__ void __launch_bounds__(256) sched_count_scatter_kernel(const SchedArgs a, int pass) {
+  __shared__ int s_key[SCHED_HASH];
+  __shared__ int s_cnt[SCHED_HASH];               // entries per bucket, then (pass 1) the bucket's base
   const int t0 = blockIdx.x * SCHED_ROWS;
   const int t1 = min(a.total_q, t0 + SCHED_ROWS);
   const int per_row = a.Hkv * a.topk;
-  const long e0 = static_cast<long>(t0) * per_row, e1 = static_cast<long>(t1) * per_row;
-  for (long e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
-    const int b = __ldg(a.block_idx + e);
-    if (b < 0) continue;
-    const int t = static_cast<int>(e / per_row);
-    const int g = static_cast<int>((e / a.topk) % a.Hkv);
-    const int slot = static_cast<int>(e % a.topk);
+  const int nent = (t1 - t0) * per_row;
+  const long e0 = static_cast<long>(t0) * per_row;
+  // the entry's bucket, or -1 (empty slot or out-of-range index, which is flagged)
+  auto bucket_of = [&](int el, int& ent) -> int {
+    const int b = __ldg(a.block_idx + e0 + el);
+    if (b < 0) return -1;
+    const int t = t0 + el / per_row;
+    const int rem = el % per_row;
+    const int g = rem / a.topk, slot = rem % a.topk;
     const int s = find_seq(a.q_start, a.num_seqs, t);
     const int qs = __ldg(a.q_start + s), nq = __ldg(a.q_start + s + 1) - qs;
     const int p = __ldg(a.ctx_len + s) - nq + (t - qs);
-    if (b >= a.max_blocks || b > p / a.block_size) { flag_error(MSA_DEV_BOUNDS); continue; }
-    const int bk = entry_bucket(a, t, g, b, s);
-    if (pass == 0) {
-      atomicAdd(&a.counts[bk], 1);
-    } else {
-      const int pos = atomicAdd(&a.cursor[bk], 1);
-      a.entries[pos] = (t << 6) | slot;
+    if (b >= a.max_blocks || b > p / a.block_size) { flag_error(MSA_DEV_BOUNDS); return -1; }
+    ent = (t << 6) | slot;
+    return entry_bucket(a, t, g, b, s);
+  };
+  if (2 * SCHED_ROWS * per_row > SCHED_HASH) {    // rows too wide for the table: one atomic per entry
+    for (int el = threadIdx.x; el < nent; el += blockDim.x) {
+      int ent = 0;
+      const int bk = bucket_of(el, ent);
+      if (bk < 0) continue;
+      if (pass == 0) atomicAdd(&a.counts[bk], 1);
+      else a.entries[atomicAdd(&a.cursor[bk], 1)] = ent;
     }
+    return;
   }
+  for (int i = threadIdx.x; i < SCHED_HASH; i += blockDim.x) { s_key[i] = -1; s_cnt[i] = 0; }
+  __syncthreads();
+  int hs[SCHED_EPT], li[SCHED_EPT], ents[SCHED_EPT];
+#pragma unroll
+  for (int k = 0; k < SCHED_EPT; ++k) {
+    hs[k] = -1;
+    li[k] = 0;
+    ents[k] = 0;
+    const int el = threadIdx.x + k * 256;
+    if (el >= nent) continue;
+    const int bk = bucket_of(el, ents[k]);
+    if (bk < 0) continue;
+    uint32_t h = (static_cast<uint32_t>(bk) * 2654435761u) >> 20;   // 12 bits
+    for (int probe = 0; probe < SCHED_HASH; ++probe) {               // the table is at most half full
+      const int prev = atomicCAS(&s_key[h], -1, bk);
+      if (prev == -1 || prev == bk) { hs[k] = static_cast<int>(h); break; }
+      h = (h + 1) & (SCHED_HASH - 1);
+    }
+    if (hs[k] >= 0) li[k] = atomicAdd(&s_cnt[hs[k]], 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < SCHED_HASH; i += blockDim.x) {
+    const int bk = s_key[i];
+    if (bk < 0) continue;
+    if (pass == 0) atomicAdd(&a.counts[bk], s_cnt[i]);
+    else s_cnt[i] = atomicAdd(&a.cursor[bk], s_cnt[i]);
+  }
+  if (pass == 0) return;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < SCHED_EPT; ++k)
+    if (hs[k] >= 0) a.entries[s_cnt[hs[k]] + li[k]] = ents[k];
 }
 
 // one CTA: exclusive scans of entry counts and of tiles per bucket, packed as
