@@ -123,6 +123,29 @@ def test_attention_matches_oracle(cuda_ok, which, path):
     assert max(lerr) <= H.LSE_MAX_ABS, max(lerr)
 
 
+def test_wide_selection_rows_match_oracle(cuda_ok):
+    """k = 32 over 4 groups: 128 entries per query row, more than the prefill schedule's per-CTA
+    bucket table holds, so its per-entry counting path builds the tiles."""
+    wl = gen.make_workload("mixed_k32", seed=8, ctx_len=[1000, 3000, 129, 5000, 256], nq=[1000, 300, 129, 200, 1],
+                           num_q_heads=64, num_kv_heads=4, idx_heads=8, topk=32, plant_frac=0.1, random_pages=True)
+    d = H.device_inputs(wl)
+    sel = _oracle_selection(wl, 13)
+    out, lse = H.run_attn(d, torch.from_numpy(sel).cuda(), "prefill")
+    assert msa.device_status() == msa.MSA_OK
+    errs, lerr = [], []
+    for s in range(wl.num_seqs):
+        rows = list(H.seq_rows(wl, s))
+        if len(rows) > 300:
+            rows = rows[:48] + rows[-48:]
+        ref, ref_lse = H.oracle_attention_rows(d, s, rows, sel[rows])
+        errs.append(H.attn_errors(out[rows], ref))
+        lerr.append(float(np.abs(lse[rows].cpu().numpy() - ref_lse).max()))
+    mx = max(e[0] for e in errs)
+    mean = float(np.mean([e[1] for e in errs]))
+    assert mx <= H.ATTN_MAX_ABS and mean <= H.ATTN_MEAN_ABS, (mx, mean)
+    assert max(lerr) <= H.LSE_MAX_ABS, max(lerr)
+
+
 def test_all_blocks_selected_is_dense_causal(cuda_ok):
     """k >= number of blocks: every row attends to its whole causal prefix."""
     wl = configs.tiny_prefill_2k()
