@@ -28,6 +28,7 @@ EXPORTS = (
     "msa_prefill_workspace_bytes", "msa_decode_workspace_bytes", "msa_get_device_status",
     "msa_set_wait_limit_ns", "msa_debug_wait_timeout", "msa_status_string", "msa_last_error",
     "msa_version", "msa_attn_decode_noalloc", "msa_index_topk", "msa_set_timing_events",
+    "msa_qknorm_rope_insert",
 )
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, MSA_ERR_DEVICE_BOUNDS = range(6)
@@ -74,6 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "msa_attn_prefill": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
         "msa_attn_decode": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
         "msa_attn_decode_noalloc": [cfgp, batp, P, P, P, P, P, P, P],
+        "msa_qknorm_rope_insert": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_float, ctypes.c_float, P],
         "msa_prefill_workspace_bytes": [cfgp, batp],
         "msa_decode_workspace_bytes": [cfgp, batp],
         "msa_get_device_status": [P],
@@ -239,6 +241,19 @@ def attn_prefill(cfg: Config, batch: Batch, q, k_cache, v_cache, block_idx, out,
 def attn_decode(cfg: Config, batch: Batch, q, k_cache, v_cache, block_idx, out, lse=None, workspace=None,
                 stream=None) -> None:
     _attn(load_library().msa_attn_decode, cfg, batch, q, k_cache, v_cache, block_idx, out, lse, workspace, stream)
+
+
+def qknorm_rope_insert(cfg: Config, batch: Batch, q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache,
+                       rotary_dim: int = 64, rope_theta: float = 10000.0, eps: float = 1e-6, stream=None) -> None:
+    """Per-head RMSNorm + partial rotary embedding of q (in place) and of the new keys, whose
+    rows go with the new values into their cache page and slot (see include/msa.h)."""
+    lib = load_library()
+    _check(lib.msa_qknorm_rope_insert(ctypes.byref(cfg._c()), ctypes.byref(batch._c()),
+                                      _need(q, torch.bfloat16, "q"), _need(k_new, torch.bfloat16, "k_new"),
+                                      _need(v_new, torch.bfloat16, "v_new"), _need(q_norm_w, torch.bfloat16, "q_norm_w"),
+                                      _need(k_norm_w, torch.bfloat16, "k_norm_w"),
+                                      _need(k_cache, torch.bfloat16, "k_cache"), _need(v_cache, torch.bfloat16, "v_cache"),
+                                      int(rotary_dim), float(rope_theta), float(eps), _stream(stream)))
 
 
 def attn_decode_noalloc(cfg: Config, batch: Batch, q, k_cache, v_cache, block_idx, out, lse=None,

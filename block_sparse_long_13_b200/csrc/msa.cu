@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "index_decode.cuh"
 #include "index_prefill.cuh"
+#include "qk_rope_insert.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -528,6 +529,48 @@ msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, 
   CUDA_TRY(cudaMemsetAsync(a.counters, 0, units * 4, stream));
   CUDA_TRY(set_smem(msa::attn_decode_kernel, msa::ATTD_SMEM));   // with the static arrays: above the 48 KiB default
   msa::attn_decode_kernel<<<static_cast<unsigned>(units * w.nsplit), msa::ATTD_THREADS, msa::ATTD_SMEM, stream>>>(a);
+  return launched();
+}
+
+msa_status_t msa_qknorm_rope_insert(const msa_config_t* cfg, const msa_batch_t* batch, void* q, const void* k_new,
+                                    const void* v_new, const void* q_norm_w, const void* k_norm_w, void* k_cache,
+                                    void* v_cache, int32_t rotary_dim, float rope_theta, float eps,
+                                    cudaStream_t stream) {
+  msa_status_t st;
+  if ((st = check_config(cfg)) != MSA_OK) return st;
+  if ((st = check_batch(batch)) != MSA_OK) return st;
+  CHECK_ARG(q && k_new && v_new && q_norm_w && k_norm_w && k_cache && v_cache,
+            "q, k_new, v_new, the norm weights and the caches must not be NULL");
+  CHECK_ARG(aligned16(q) && aligned16(k_new) && aligned16(v_new) && aligned16(q_norm_w) && aligned16(k_norm_w) &&
+                aligned16(k_cache) && aligned16(v_cache),
+            "pointers must be 16-byte aligned");
+  CHECK_ARG(rotary_dim > 0 && rotary_dim % 8 == 0 && rotary_dim <= cfg->head_dim,
+            "rotary_dim must be a positive multiple of 8, at most head_dim");
+  CHECK_ARG(std::isfinite(rope_theta) && rope_theta > 0.f, "rope_theta must be positive and finite");
+  CHECK_ARG(std::isfinite(eps) && eps >= 0.f, "eps must be finite and >= 0");
+  if (batch->total_q == 0) return MSA_OK;
+  msa::QkRopeArgs a{};
+  a.q = static_cast<__nv_bfloat16*>(q);
+  a.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  a.q_w = static_cast<const __nv_bfloat16*>(q_norm_w);
+  a.k_w = static_cast<const __nv_bfloat16*>(k_norm_w);
+  a.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  a.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  a.q_start = batch->q_start;
+  a.ctx_len = batch->ctx_len;
+  a.page_table = batch->page_table;
+  a.num_seqs = batch->num_seqs;
+  a.total_q = batch->total_q;
+  a.Hq = cfg->num_q_heads;
+  a.Hkv = cfg->num_kv_heads;
+  a.max_blocks = batch->max_blocks_per_seq;
+  a.num_pages = batch->num_pages;
+  a.block_size = cfg->block_size;
+  a.rotary_dim = rotary_dim;
+  a.log2_theta = std::log2(static_cast<double>(rope_theta));
+  a.eps = eps;
+  msa::qk_rope_insert_kernel<<<static_cast<unsigned>(batch->total_q), msa::QKR_THREADS, 0, stream>>>(a);
   return launched();
 }
 

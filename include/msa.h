@@ -193,6 +193,37 @@ msa_status_t msa_attn_decode_noalloc(const msa_config_t* cfg, const msa_batch_t*
                                      const void* k_cache, const void* v_cache, const int32_t* block_idx, void* out,
                                      float* lse, cudaStream_t stream);
 
+/*
+ * The step just before the path, fused: per-head QK normalization, partial
+ * rotary embedding and the paged K/V insert of this call's new rows
+ * ("MiniMax-M3", inteligile model page, table "Checked in its code", rows
+ * "QK normalization" and "Partial RoPE"; daily.dev "MiniMax M3 ...", section
+ * "Serving options": fused QKNorm + RoPE + KV insert).  For every new row t of
+ * sequence s at absolute position p = ctx_len[s] - n_q(s) + i (the i-th of the
+ * sequence's n_q new rows):
+ *   q[t][h]                                 = rope(rmsnorm(q[t][h]) * q_norm_w)   (in place)
+ *   k_cache[page][g][p % block_size][:]     = rope(rmsnorm(k_new[t][g]) * k_norm_w)
+ *   v_cache[page][g][p % block_size][:]     = v_new[t][g],   page = page_table[s][p / block_size]
+ * rmsnorm(x) = x / sqrt(mean over the head's head_dim channels of x^2 + eps);
+ * rope turns channel pairs (i, i + rotary_dim/2), i < rotary_dim/2, by the
+ * angle p * rope_theta^(-2i / rotary_dim) (first of the pair: a cos - b sin,
+ * second: b cos + a sin); channels from rotary_dim on pass through.  The pages
+ * fix rotary_dim = 64 of 128; they give neither rope_theta nor eps, so both are
+ * arguments.  Angles are formed in double precision.
+ *   q         bf16 [total_q][num_q_heads][head_dim], read and overwritten
+ *   k_new     bf16 [total_q][num_kv_heads][head_dim]   (v_new alike)
+ *   q_norm_w  bf16 [head_dim], shared by the query heads (k_norm_w: key heads)
+ *   k_cache   bf16 [num_pages][num_kv_heads][block_size][head_dim] (v_cache alike)
+ * rotary_dim must be a positive multiple of 8, at most head_dim.  A page id
+ * outside [0, num_pages) is recorded as MSA_ERR_DEVICE_BOUNDS and that row's
+ * cache writes are skipped (its queries are still written).  k_new and v_new
+ * must not overlap the caches or q.
+ */
+msa_status_t msa_qknorm_rope_insert(const msa_config_t* cfg, const msa_batch_t* batch, void* q, const void* k_new,
+                                    const void* v_new, const void* q_norm_w, const void* k_norm_w, void* k_cache,
+                                    void* v_cache, int32_t rotary_dim, float rope_theta, float eps,
+                                    cudaStream_t stream);
+
 /* Timing hook (no counterpart on the pages).  With n = 4 and four cudaEvent_t
  * handles (owned by the caller), every later msa_attn_prefill call on this host
  * thread records events[0] before its schedule kernels, events[1] before the

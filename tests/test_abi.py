@@ -121,6 +121,28 @@ def test_fused_index_topk_checks(lib):
     assert lib.msa_index_topk(ctypes.byref(bad), ctypes.byref(b), p, p, p, None) == msa.MSA_ERR_UNSUPPORTED
 
 
+def test_qknorm_rope_insert_checks(lib):
+    """Argument checks of the fused norm / rotary / insert call (nothing is launched)."""
+    b = _batch()._c(host_only=True)
+    p = ctypes.c_void_p(16)
+    cfg = msa.Config()._c()
+    def call(rd=64, theta=10000.0, eps=1e-6, ptrs=None):
+        a = ptrs or [p] * 7
+        return lib.msa_qknorm_rope_insert(ctypes.byref(cfg), ctypes.byref(b), *a, rd, theta, eps, None)
+    for rd in (0, -8, 60, 136):
+        assert call(rd=rd) == msa.MSA_ERR_INVALID_ARG, rd
+    assert b"rotary_dim" in lib.msa_last_error()
+    assert call(theta=0.0) == msa.MSA_ERR_INVALID_ARG
+    assert call(theta=float("inf")) == msa.MSA_ERR_INVALID_ARG
+    assert call(eps=-1.0) == msa.MSA_ERR_INVALID_ARG
+    assert call(eps=float("nan")) == msa.MSA_ERR_INVALID_ARG
+    assert call(ptrs=[p] * 6 + [None]) == msa.MSA_ERR_INVALID_ARG
+    assert call(ptrs=[p] * 3 + [ctypes.c_void_p(24)] + [p] * 3) == msa.MSA_ERR_INVALID_ARG
+    bad = _cfg(head_dim=64)._c()
+    assert lib.msa_qknorm_rope_insert(ctypes.byref(bad), ctypes.byref(b), *([p] * 7), 64, 10000.0, 1e-6, None) == \
+        msa.MSA_ERR_UNSUPPORTED
+
+
 def test_timing_events_hook_checks(lib):
     assert lib.msa_set_timing_events(None, 3) == msa.MSA_ERR_INVALID_ARG
     assert lib.msa_set_timing_events(None, 4) == msa.MSA_ERR_INVALID_ARG
