@@ -192,6 +192,46 @@ def build_parts(name, batch=None, fused=False):
     return parts
 
 
+# ------------------------------------------------------------------ next rows, timed on their own
+
+def time_next_rows(parts, pk):
+    """The fused QK-norm + partial-RoPE + KV-insert call (the step just before the path) on the
+    workload's first prefill chunk, timed by itself: it is not part of the step, whose inputs are
+    already normed, rotated and inserted.  Algorithmic bytes per row: q read and written in place,
+    the new k and v rows read and written to the cache."""
+    import block_sparse_long_13_b200 as msa
+    p = next((x for x in parts if x.kind == "prefill"), None)
+    if p is None:
+        return None
+    wl = p.wl
+    T, hq, hkv, d = wl.total_q, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
+    q = p.q.clone()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    kn = torch.randn((T, hkv, d), device="cuda", generator=g).to(torch.bfloat16)
+    vn = torch.randn((T, hkv, d), device="cuda", generator=g).to(torch.bfloat16)
+    w = torch.ones(d, device="cuda", dtype=torch.bfloat16)
+    kc, vc = p.caches["k"].clone(), p.caches["v"].clone()
+
+    def call():
+        msa.qknorm_rope_insert(p.cfg, p.batch, q, kn, vn, w, w, kc, vc)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 20
+    e0.record()
+    for _ in range(n):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    nbytes = T * 2 * (hq + 2 * hkv) * d * 2
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"qk_rope_insert_kernel": {"part": p.name, "rows": T, "ms_per_call": ms, "bytes_per_call": nbytes,
+                                      "gbs": gbs, "frac": gbs / pk["hbm_gbs"], "status": int(msa.device_status())}}
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -582,6 +622,14 @@ def main():
                "d2h_bytes_per_step": int(d2h), "ms_per_step": ems}
     st = msa.device_status()
 
+    # never let this extra measurement cost the line itself
+    next_rows = None
+    if rank == 0:
+        try:
+            next_rows = time_next_rows(parts, pk)
+        except Exception as exc:  # noqa: BLE001
+            next_rows = {"error": str(exc)[:200]}
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample()
@@ -596,7 +644,7 @@ def main():
                 "roofline": roof, "fractions": fractions, "parts": parts_summary,
                 "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
                 "gpu_launches": sum(p.launches for p in parts) * args.steps,
-                "device_status": int(st)}
+                "device_status": int(st), "next_rows": next_rows}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
