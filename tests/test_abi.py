@@ -106,6 +106,22 @@ def test_bad_batch_and_pointers_rejected(lib):
     assert lib.msa_set_wait_limit_ns(0) == msa.MSA_ERR_INVALID_ARG
 
 
+def test_empty_batch_launches_nothing(lib):
+    """total_q = 0 (a sequence with no new rows): every compute call checks its arguments and
+    returns MSA_OK without launching; on a machine without a GPU any launch would fail."""
+    cfg = msa.Config()._c()
+    b = msa.Batch.make([0, 0], [300], [list(range(3))], 3, device="cpu")._c(host_only=True)
+    p = ctypes.c_void_p(16)
+    n = 1 << 20
+    assert lib.msa_index_scores(ctypes.byref(cfg), ctypes.byref(b), p, p, p, None) == msa.MSA_OK
+    assert lib.msa_topk_blocks(ctypes.byref(cfg), ctypes.byref(b), p, p, None) == msa.MSA_OK
+    assert lib.msa_index_topk(ctypes.byref(cfg), ctypes.byref(b), p, p, p, None) == msa.MSA_OK
+    assert lib.msa_attn_prefill(ctypes.byref(cfg), ctypes.byref(b), p, p, p, p, p, None, p, n, None) == msa.MSA_OK
+    assert lib.msa_attn_decode(ctypes.byref(cfg), ctypes.byref(b), p, p, p, p, p, None, p, n, None) == msa.MSA_OK
+    assert lib.msa_qknorm_rope_insert(ctypes.byref(cfg), ctypes.byref(b), *([p] * 7), 64, 10000.0, 1e-6,
+                                      None) == msa.MSA_OK
+
+
 def test_fused_index_topk_checks(lib):
     """The fused call validates like the two calls it replaces and keeps at most 16 blocks per row."""
     b = _batch()._c(host_only=True)
