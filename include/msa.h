@@ -32,6 +32,10 @@
  *     declared) and bounded waits that ran out are recorded in a device error
  *     word and reported by msa_get_device_status(); the kernels skip the bad
  *     access instead of faulting.
+ *   - Cache slots of a page past a sequence's ctx_len (the unwritten tail of
+ *     its last page) must hold finite values: the tensor-core P.V multiplies
+ *     those V rows by zero probabilities, and 0 * NaN is NaN.  Pages that come
+ *     zeroed or hold earlier finite writes satisfy this.
  *
  * LAYOUTS (row-major, bf16 = IEEE bfloat16, fp32 = IEEE float)
  *   idx_q        bf16 [total_q][idx_heads][idx_dim]
