@@ -28,7 +28,7 @@ EXPORTS = (
     "msa_prefill_workspace_bytes", "msa_decode_workspace_bytes", "msa_get_device_status",
     "msa_set_wait_limit_ns", "msa_debug_wait_timeout", "msa_status_string", "msa_last_error",
     "msa_version", "msa_attn_decode_noalloc", "msa_index_topk", "msa_set_timing_events",
-    "msa_qknorm_rope_insert",
+    "msa_qknorm_rope_insert", "msa_merge_partials",
 )
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, MSA_ERR_DEVICE_BOUNDS = range(6)
@@ -76,6 +76,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "msa_attn_decode": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_size_t, P],
         "msa_attn_decode_noalloc": [cfgp, batp, P, P, P, P, P, P, P],
         "msa_qknorm_rope_insert": [cfgp, batp, P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_float, ctypes.c_float, P],
+        "msa_merge_partials": [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, P, P, P, P, P],
         "msa_prefill_workspace_bytes": [cfgp, batp],
         "msa_decode_workspace_bytes": [cfgp, batp],
         "msa_get_device_status": [P],
@@ -254,6 +255,16 @@ def qknorm_rope_insert(cfg: Config, batch: Batch, q, k_new, v_new, q_norm_w, k_n
                                       _need(k_norm_w, torch.bfloat16, "k_norm_w"),
                                       _need(k_cache, torch.bfloat16, "k_cache"), _need(v_cache, torch.bfloat16, "v_cache"),
                                       int(rotary_dim), float(rope_theta), float(eps), _stream(stream)))
+
+
+def merge_partials(outs, lses, out, lse=None, stream=None) -> None:
+    """Log-sum-exp merge of n partials: outs bf16 [n][..][128], lses fp32 [n][..] -> out, lse."""
+    n = int(outs.shape[0])
+    units = int(lses[0].numel())
+    lib = load_library()
+    _check(lib.msa_merge_partials(n, units, int(outs.shape[-1]), _need(outs, torch.bfloat16, "outs"),
+                                  _need(lses, torch.float32, "lses"), _need(out, torch.bfloat16, "out"),
+                                  _need(lse, torch.float32, "lse"), _stream(stream)))
 
 
 def attn_decode_noalloc(cfg: Config, batch: Batch, q, k_cache, v_cache, block_idx, out, lse=None,

@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "index_decode.cuh"
 #include "index_prefill.cuh"
+#include "merge_partials.cuh"
 #include "qk_rope_insert.cuh"
 #include "topk.cuh"
 
@@ -571,6 +572,24 @@ msa_status_t msa_qknorm_rope_insert(const msa_config_t* cfg, const msa_batch_t* 
   a.log2_theta = std::log2(static_cast<double>(rope_theta));
   a.eps = eps;
   msa::qk_rope_insert_kernel<<<static_cast<unsigned>(batch->total_q), msa::QKR_THREADS, 0, stream>>>(a);
+  return launched();
+}
+
+msa_status_t msa_merge_partials(int32_t n, int64_t units, int32_t head_dim, const void* outs, const float* lses,
+                                void* out, float* lse, cudaStream_t stream) {
+  CHECK_ARG(n >= 1 && n <= 4096, "n must be in [1, 4096]");
+  CHECK_ARG(units >= 0, "units must be >= 0");
+  CHECK_SUP(head_dim == 128, "head_dim must be 128");
+  CHECK_ARG(outs && lses && out, "outs, lses and out must not be NULL");
+  CHECK_ARG(aligned16(outs) && aligned16(out) && (reinterpret_cast<uintptr_t>(lses) & 3u) == 0 &&
+                (reinterpret_cast<uintptr_t>(lse) & 3u) == 0,
+            "outs and out must be 16-byte aligned, lses and lse 4-byte aligned");
+  if (units == 0) return MSA_OK;
+  const long warps_per_cta = msa::MRG_THREADS / 32;
+  const long grid = (units + warps_per_cta - 1) / warps_per_cta;
+  CHECK_SUP(grid <= 0x7FFFFFFFL, "too many rows");
+  msa::merge_partials_kernel<<<static_cast<unsigned>(grid), msa::MRG_THREADS, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(outs), lses, static_cast<__nv_bfloat16*>(out), lse, n, units);
   return launched();
 }
 

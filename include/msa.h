@@ -228,6 +228,20 @@ msa_status_t msa_qknorm_rope_insert(const msa_config_t* cfg, const msa_batch_t* 
                                     void* v_cache, int32_t rotary_dim, float rope_theta, float eps,
                                     cudaStream_t stream);
 
+/*
+ * Log-sum-exp merge of n partial attentions over disjoint key sets ("LSE
+ * fusion", "Two-phase forward": inteligile "MiniMax-M3" model page, tags), as
+ * needed to join the results of one sequence whose KV blocks sit on several
+ * GPUs:  L = log sum_s exp(lse_s),  out = sum_s exp(lse_s - L) out_s.
+ *   outs  bf16 [n][units][head_dim]   each partial normalised over its own keys
+ *   lses  fp32 [n][units]             natural log; -inf = the partial saw no key (weight 0)
+ *   out   bf16 [units][head_dim]      lse fp32 [units] (L), or NULL
+ * units = rows x heads; head_dim must be 128.  Rows whose partials are all
+ * -inf get out = 0 and lse = -inf.
+ */
+msa_status_t msa_merge_partials(int32_t n, int64_t units, int32_t head_dim, const void* outs, const float* lses,
+                                void* out, float* lse, cudaStream_t stream);
+
 /* Timing hook (no counterpart on the pages).  With n = 4 and four cudaEvent_t
  * handles (owned by the caller), every later msa_attn_prefill call on this host
  * thread records events[0] before its schedule kernels, events[1] before the

@@ -159,6 +159,16 @@ def test_qknorm_rope_insert_checks(lib):
         msa.MSA_ERR_UNSUPPORTED
 
 
+def test_merge_partials_checks(lib):
+    p, f = ctypes.c_void_p(16), ctypes.c_void_p(20)
+    assert lib.msa_merge_partials(0, 8, 128, p, p, p, None, None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_merge_partials(2, -1, 128, p, p, p, None, None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_merge_partials(2, 8, 64, p, p, p, None, None) == msa.MSA_ERR_UNSUPPORTED
+    assert lib.msa_merge_partials(2, 8, 128, None, p, p, None, None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_merge_partials(2, 8, 128, f, p, p, None, None) == msa.MSA_ERR_INVALID_ARG   # outs misaligned
+    assert lib.msa_merge_partials(2, 0, 128, p, f, p, f, None) == msa.MSA_OK                  # nothing to merge
+
+
 def test_timing_events_hook_checks(lib):
     assert lib.msa_set_timing_events(None, 3) == msa.MSA_ERR_INVALID_ARG
     assert lib.msa_set_timing_events(None, 4) == msa.MSA_ERR_INVALID_ARG
