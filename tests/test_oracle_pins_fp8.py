@@ -67,3 +67,24 @@ def test_scores_from_dequantized_keys_brute_force():
             want = -math.inf if not js else sum(max(sum(q[t, h, c] * kd[j, h, c] for c in range(4)) for j in js)
                                                 for h in range(H))
             assert (got[t, 0, b] == want) if want == -math.inf else abs(got[t, 0, b] - want) <= 1e-12
+
+
+def test_pins_catch_plausible_slips():
+    """Rounding ties away from zero, truncating, or letting values past 448 through would each
+    break a pin above."""
+    x = np.array([1.0625, 1.1875, 3.0625, 2 ** -10, 3 * 2 ** -10, 460.0, 1e6])
+    want = torch.from_numpy(np.clip(x, -448, 448)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+    def rounded(y, mode):
+        a = np.abs(y)
+        _, e = np.frexp(a)
+        e = np.maximum(e - 1, -6)
+        qn = np.ldexp(1.0, e - 3)
+        m = a / qn
+        r = {"away": np.floor(m + 0.5), "trunc": np.floor(m)}[mode]
+        return np.copysign(r * qn, y)
+
+    assert np.array_equal(F.round_e4m3(x), want)
+    assert not np.array_equal(rounded(np.clip(x, -448, 448), "away"), want)
+    assert not np.array_equal(rounded(np.clip(x, -448, 448), "trunc"), want)
+    assert F.round_e4m3(np.array([1e6]))[0] == 448.0 != rounded(np.array([1e6]), "away")[0]

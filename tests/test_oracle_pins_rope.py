@@ -111,3 +111,38 @@ def test_insert_writes_exactly_the_rows_of_the_call():
     np.testing.assert_allclose(kc2, kexp, rtol=0, atol=1e-12)
     np.testing.assert_array_equal(vc2, vexp)
     assert q_out.shape == q.shape
+
+
+def test_fixtures_catch_plausible_slips():
+    """The hand-worked cases fail for the slips a restatement could make: interleaved pairs
+    (i, i+1) instead of (i, i + r/2), the rotation turned the other way, eps outside the root,
+    and the frequency exponent -i/r instead of -2i/r."""
+    with open(os.path.join(GOLD, "qknorm_rope_handworked.json")) as f:
+        g = json.load(f)
+
+    def norm(x, w, eps, outside=False):
+        ms = np.mean(x * x)
+        return (x / (np.sqrt(ms) + eps) if outside else x / np.sqrt(ms + eps)) * np.asarray(w, dtype=np.float64)
+
+    def rope(x, p, r, theta, pairing="half", sign=1.0, expo=2.0):
+        y = x.copy()
+        for i in range(r // 2):
+            a_i, b_i = (i, i + r // 2) if pairing == "half" else (2 * i, 2 * i + 1)
+            ang = sign * p * theta ** (-expo * i / r)
+            a, b = x[a_i], x[b_i]
+            y[a_i], y[b_i] = a * math.cos(ang) - b * math.sin(ang), b * math.cos(ang) + a * math.sin(ang)
+        return y
+
+    def run(c, **kw):
+        outside = kw.pop("outside", False)
+        x = np.array(c["x"], dtype=np.float64)
+        return rope(norm(x, c["w"], c["eps"], outside), c["pos"], c["rotary_dim"], c["theta"], **kw)
+
+    def matches_all(**kw):
+        return all(np.allclose(run(c, **dict(kw)), c["expected"], atol=1e-9) for c in g["cases"])
+
+    assert matches_all()                                  # the restatement itself reproduces every case
+    assert not matches_all(pairing="interleaved")
+    assert not matches_all(sign=-1.0)
+    assert not matches_all(outside=True)
+    assert not matches_all(expo=1.0)
