@@ -115,7 +115,7 @@ def _worker(rank, ws, port, ctx, seed, qout):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("ws,ctx", [(2, 1500), (3, 1500), (3, 200)])
+@pytest.mark.parametrize("ws,ctx", [(2, 1500), (3, 1500), (3, 200), (1, 1500), (2, 1536), (3, 1537)])
 def test_context_parallel_decode_matches_single_process(ws, ctx):
     c = mp.get_context("spawn")
     q = c.Queue()
