@@ -47,8 +47,13 @@ def peaks():
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
                 "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
-                "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+                "source": "measured", **SPEC}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback", **SPEC}
+
+
+# nominal B200 figures the per-workload fractions are also stated against: 8 TB/s of HBM (the
+# decode target's denominator) and 2.25 PFLOP/s of dense bf16
+SPEC = {"hbm_gbs_spec": 8000.0, "bf16_tflops_spec": 2250.0}
 
 
 def recorded_traffic(kernel):
@@ -190,6 +195,74 @@ def build_parts(name, batch=None, fused=False):
                   "idx_k": gen.paged_cache(wl, gen.TID_IDX_K, device="cuda")}
         parts.append(Part(name, wl, caches, "prefill", fused=fused))
     return parts
+
+
+# ------------------------------------------------------------------ per-call times and per-workload fractions
+
+def call_stats(parts, evs, steps, stop_after="attn"):
+    """Per part: device time of each call (mean over the timed steps, CUDA events on the
+    launching stream) and its algorithmic work."""
+    calls = {}
+    for i, p in enumerate(parts):
+        t_idx = statistics.mean(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(steps))
+        t_top = statistics.mean(evs[k][i][1].elapsed_time(evs[k][i][2]) for k in range(steps))
+        t_att = statistics.mean(evs[k][i][2].elapsed_time(evs[k][i][3]) for k in range(steps))
+        phase = None
+        if p.kind == "prefill" and stop_after == "attn":
+            phase = {nm: statistics.mean(evs[k][i][4 + j].elapsed_time(evs[k][i][5 + j]) for k in range(steps))
+                     for j, nm in enumerate(("schedule_ms", "kernel_ms", "merge_ms"))}
+        calls[p.name] = {"index_ms": t_idx, "topk_ms": t_top, "attn_ms": t_att, "attn_phases": phase,
+                         "index": p.index_work(), "attn": p.attn_work(), "topk": p.topk_work(), "kind": p.kind,
+                         "merge": p.merge_work() if p.kind == "prefill" else None,
+                         "tokens": p.wl.total_q, "fused": p.fused}
+    return calls
+
+
+def workload_summary(calls, pk):
+    """Fractions of the roofline per workload, as the decode and prefill targets state them:
+    prefill = (indexer causal FLOPs + attention FLOPs) / (indexer + top-k + attention time) over
+    the dense bf16 peak (measured burst and nominal 2.25 PF; attention-only and indexer-only
+    beside); decode = (indexer-key bytes + visible selected K/V + q/out) / (indexer + top-k +
+    attention time) over 8 TB/s and over the measured copy bandwidth."""
+    cs = list(calls.values())
+    ms = sum(c["index_ms"] + c["topk_ms"] + c["attn_ms"] for c in cs)
+    tokens = sum(c["tokens"] for c in cs)
+    r = {"tokens": tokens, "ms": ms, "tokens_per_s": tokens / (ms / 1e3)}
+    if cs[0]["kind"] == "prefill":
+        fi = sum(c["index"]["flops"] for c in cs)
+        fa = sum(c["attn"]["flops"] for c in cs)
+        tf = (fi + fa) / ms / 1e9
+        ti = sum(c["index_ms"] for c in cs)
+        ta = sum(c["attn_ms"] for c in cs)
+        r.update(index_tflop=fi / 1e12, attn_tflop=fa / 1e12, tflops=tf,
+                 frac_dense_measured=tf / pk["bf16_tflops"], frac_dense_spec=tf / pk["bf16_tflops_spec"],
+                 attn_only_frac_measured=(fa / ta / 1e9) / pk["bf16_tflops"] if ta > 0 else None,
+                 index_only_frac_measured=(fi / ti / 1e9) / pk["bf16_tflops"] if ti > 0 else None)
+    else:
+        b = sum(c["index"]["bytes"] + c["attn"]["bytes"] for c in cs)
+        gbs = b / ms / 1e6
+        r.update(gbytes=b / 1e9, gbs=gbs, frac_hbm_8tbs=gbs / pk["hbm_gbs_spec"],
+                 frac_hbm_measured=gbs / pk["hbm_gbs"])
+    return r
+
+
+def time_workload(name, workspace, steps=3, warmup=2):
+    """A further workload timed on its own after the step (same calls, same timing method);
+    returns its summary, or an error note."""
+    parts = build_parts(name)
+    need = max(p.ws_bytes for p in parts)
+    ws = workspace if workspace.numel() >= need else torch.empty(need, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        for p in parts:
+            p.run(ws, None, stream)
+    torch.cuda.synchronize()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in parts] for _ in range(steps)]
+    for k in range(steps):
+        for i, p in enumerate(parts):
+            p.run(ws, evs[k][i], stream)
+    torch.cuda.synchronize()
+    return parts, call_stats(parts, evs, steps)
 
 
 # ------------------------------------------------------------------ next rows, timed on their own
@@ -392,6 +465,7 @@ def main():
                     help="profiling: run the step only up to this call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the 32K prefill and ragged verify timings")
     ap.add_argument("--fused-prefill", action="store_true",
                     help="prefill indexer and top-k in one call (msa_index_topk) instead of the two calls")
     args = ap.parse_args()
@@ -446,19 +520,7 @@ def main():
     value = job_throughput(tokens, ws, ms_max)
 
     # per-call device times (average over the timed steps) and algorithmic work
-    calls = {}
-    for i, p in enumerate(parts):
-        t_idx = statistics.mean(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps))
-        t_top = statistics.mean(evs[k][i][1].elapsed_time(evs[k][i][2]) for k in range(args.steps))
-        t_att = statistics.mean(evs[k][i][2].elapsed_time(evs[k][i][3]) for k in range(args.steps))
-        phase = None
-        if p.kind == "prefill" and args.stop_after == "attn":
-            phase = {nm: statistics.mean(evs[k][i][4 + j].elapsed_time(evs[k][i][5 + j]) for k in range(args.steps))
-                     for j, nm in enumerate(("schedule_ms", "kernel_ms", "merge_ms"))}
-        calls[p.name] = {"index_ms": t_idx, "topk_ms": t_top, "attn_ms": t_att, "attn_phases": phase,
-                         "index": p.index_work(), "attn": p.attn_work(), "topk": p.topk_work(), "kind": p.kind,
-                         "merge": p.merge_work() if p.kind == "prefill" else None,
-                         "tokens": p.wl.total_q, "fused": p.fused}
+    calls = call_stats(parts, evs, args.steps, args.stop_after)
     pk = peaks()
     # per kernel: device time per step (CUDA events on the launching stream) and algorithmic work
     kern = {}
@@ -486,8 +548,9 @@ def main():
             addk("index_decode_kernel", c["index_ms"], 1, bytes_=c["index"]["bytes"])
             addk("topk kernel (decode)", c["topk_ms"], 1, bytes_=c["topk"]["bytes"])
             addk("attn_decode_kernel", c["attn_ms"], 1, bytes_=c["attn"]["bytes"])
-    # every kernel is timed inside a step of tens of ms: the sustained tensor peak is the denominator
-    tensor_peak, tensor_src = pk["bf16_tflops_sustained"], pk["source"] + " sustained bf16 (cuBLAS, power-capped)"
+    # every kernel is timed inside a step of tens of ms, far shorter than the seconds-long loop the
+    # sustained figure comes from: the burst tensor peak is the denominator
+    tensor_peak, tensor_src = pk["bf16_tflops"], pk["source"] + " burst bf16 (cuBLAS)"
     fractions = {}
     for name, k in kern.items():
         if k["ms"] <= 0:
@@ -517,15 +580,12 @@ def main():
                 "frac": ach / pk["hbm_gbs"], "traffic": traffic, "peak_source": pk["source"] + " copy",
                 "launch_ms": launch_ms, "bytes_per_launch": dom["bytes"] / dom["launches"]}
     parts_summary = {}
-    pre = [c for c in calls.values() if c["kind"] == "prefill"]
+    pre = {n: c for n, c in calls.items() if c["kind"] == "prefill"}
     if pre:
-        t = sum(c["index_ms"] + c["topk_ms"] + c["attn_ms"] for c in pre)
-        parts_summary["prefill"] = {"tokens": sum(c["tokens"] for c in pre), "ms": t,
-                                    "tokens_per_s": sum(c["tokens"] for c in pre) / (t / 1e3)}
+        parts_summary["prefill"] = workload_summary(pre, pk)
     for name, c in calls.items():
         if c["kind"] == "decode":
-            t = c["index_ms"] + c["topk_ms"] + c["attn_ms"]
-            parts_summary[name] = {"tokens": c["tokens"], "ms": t, "tokens_per_s": c["tokens"] / (t / 1e3)}
+            parts_summary[name] = workload_summary({name: c}, pk)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -629,6 +689,17 @@ def main():
             next_rows = time_next_rows(parts, pk)
         except Exception as exc:  # noqa: BLE001
             next_rows = {"error": str(exc)[:200]}
+
+    # the other workloads of the parity set, timed on their own after the step (not in `value`)
+    if rank == 0 and args.workload == "msa_128k_1m" and not args.no_extra:
+        for xname in ("prefill_32k", "verify_ragged"):
+            try:
+                xparts, xcalls = time_workload(xname, workspace)
+                parts_summary[xname] = dict(workload_summary(xcalls, pk), separate_run=True)
+                del xparts
+            except Exception as exc:  # noqa: BLE001
+                parts_summary[xname] = {"error": str(exc)[:200]}
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

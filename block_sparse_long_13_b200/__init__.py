@@ -258,9 +258,22 @@ def qknorm_rope_insert(cfg: Config, batch: Batch, q, k_new, v_new, q_norm_w, k_n
 
 
 def merge_partials(outs, lses, out, lse=None, stream=None) -> None:
-    """Log-sum-exp merge of n partials: outs bf16 [n][..][128], lses fp32 [n][..] -> out, lse."""
+    """Log-sum-exp merge of n partials: outs bf16 [n][..][128], lses fp32 [n][..] -> out, lse.
+
+    The kernel trusts the sizes it is given, so every shape is checked here:
+    outs must be [n, *lses.shape[1:], head_dim], out must hold units * head_dim
+    elements and lse (when given) units, units = lses[0].numel()."""
+    if outs.dim() < 2 or lses.dim() < 1 or int(lses.shape[0]) != int(outs.shape[0]):
+        raise MsaError(MSA_ERR_INVALID_ARG, "outs must be [n][..][head_dim] and lses [n][..] with the same n")
     n = int(outs.shape[0])
     units = int(lses[0].numel())
+    if tuple(outs.shape) != (n, *lses.shape[1:], int(outs.shape[-1])):
+        raise MsaError(MSA_ERR_INVALID_ARG,
+                       f"outs has shape {tuple(outs.shape)}, expected {(n, *lses.shape[1:], int(outs.shape[-1]))}")
+    if out.numel() != units * int(outs.shape[-1]):
+        raise MsaError(MSA_ERR_INVALID_ARG, f"out holds {out.numel()} elements, expected {units * int(outs.shape[-1])}")
+    if lse is not None and lse.numel() != units:
+        raise MsaError(MSA_ERR_INVALID_ARG, f"lse holds {lse.numel()} elements, expected {units}")
     lib = load_library()
     _check(lib.msa_merge_partials(n, units, int(outs.shape[-1]), _need(outs, torch.bfloat16, "outs"),
                                   _need(lses, torch.float32, "lses"), _need(out, torch.bfloat16, "out"),

@@ -636,10 +636,15 @@ void* g_noalloc_addr[kNoAllocMaxDevices] = {};
 // Device address of the array on the current device.  In host code the name
 // g_noalloc_scratch only stands for the symbol; the first call on each device
 // asks the runtime for the real address (cudaGetSymbolAddress) and keeps it.
-msa_status_t noalloc_scratch(void** out) {
+// The address belongs to the current device, so `stream` must belong to it too.
+msa_status_t noalloc_scratch(cudaStream_t stream, void** out) {
   int dev = -1;
   CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MSA_ERR_UNSUPPORTED, "device %d out of range", dev);
+  int sdev = dev;
+  CUDA_TRY(cudaStreamGetDevice(stream, &sdev));
+  if (sdev != dev)
+    return fail(MSA_ERR_INVALID_ARG, "the stream belongs to device %d but device %d is current", sdev, dev);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (g_noalloc_addr[dev] == nullptr) {
     void* p = nullptr;
@@ -664,7 +669,7 @@ extern "C" msa_status_t msa_attn_decode_noalloc(const msa_config_t* cfg, const m
                 "msa_attn_decode_noalloc; split the batch or use msa_attn_decode with a workspace",
                 need, kNoAllocScratchBytes);
   void* scratch = nullptr;
-  if ((st = noalloc_scratch(&scratch)) != MSA_OK) return st;
+  if ((st = noalloc_scratch(stream, &scratch)) != MSA_OK) return st;
   // the decode path clears its counters itself (cudaMemsetAsync, no allocation)
   return msa_attn_decode(cfg, batch, q, k_cache, v_cache, block_idx, out, lse, scratch, kNoAllocScratchBytes,
                          stream);

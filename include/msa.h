@@ -187,7 +187,11 @@ msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, 
  *     are rejected with MSA_ERR_UNSUPPORTED and a message; nothing is launched.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) and remembers it; make that first call before any
- *     stream capture.
+ *     stream capture.  The remembered address dies with the device's primary
+ *     context: do not call this entry point again in a process that has reset
+ *     the device (cudaDeviceReset).
+ *   - `stream` must belong to the current device (MSA_ERR_INVALID_ARG
+ *     otherwise), whose copy of the array the call uses.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents; the call clears the counters it needs.  Calls that can overlap
  *     on the GPU (different streams, or concurrent host threads) race on the
