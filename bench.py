@@ -355,48 +355,181 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the oracle (CPU baseline / reference arm)
 
-def oracle_sample(seconds_target=15.0, max_rows=None):
-    """Time the CPU oracle on query rows drawn uniformly from the step's
-    131,072 prefill queries (the step's 72 decode rows are 0.05% of its
-    tokens).  Inputs come from the seeded generator (on the GPU when there is
-    one, untimed) and are copied to host memory; the timed part is the oracle
-    alone: indexer over every visible block, top-k, sparse attention."""
-    from oracle import msa_oracle as O
+def cpu_model():
     try:
-        from threadpoolctl import threadpool_info
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
-    except Exception:
-        cores = 1
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    chunks = configs.chunked_prefill_128k()
-    full = chunks[-1]
-    L = full.ctx_len[0]
-    host = {}
-    for key, tid in (("idx_k", gen.TID_IDX_K), ("k", gen.TID_K), ("v", gen.TID_V)):
-        host[key] = gen.token_tensor(full, tid, 0, torch.arange(L), device=dev).float().cpu().numpy()
-    rng = np.random.default_rng(0)
-    picks = sorted(int(x) for x in rng.integers(0, L, size=512))
-    qrows = {}
-    done = 0
-    t_oracle = 0.0
-    for gpos in picks:
-        c = gpos // 16384
-        wl = chunks[c]
-        r = gpos - c * 16384
-        if c not in qrows:
-            qrows[c] = (gen.query_rows(wl, gen.TID_Q, device=dev).cpu(), gen.query_rows(wl, gen.TID_IDX_Q, device=dev).cpu())
-        q_all, iq_all = qrows[c]
-        pos = np.array([gpos])
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class _Blocks:
+    """Token-order view of one sequence of a paged device cache: slices of whole blocks (or parts
+    of one) are fetched page by page as float32 host arrays (bf16 values widened exactly)."""
+
+    def __init__(self, cache, pages, bs=128):
+        self.cache, self.pages, self.bs = cache, [int(x) for x in pages], bs
+
+    def __getitem__(self, sl):
+        b = sl.start // self.bs
+        x = self.cache[self.pages[b]].permute(1, 0, 2).float().cpu().numpy()   # [bs][H][D]
+        return x[sl.start - b * self.bs:sl.stop - b * self.bs]
+
+
+def _seq_tokens(wl, tid, s, cache=None, dev="cpu"):
+    """float32 [ctx][H][D] of one sequence in token order: from the device cache when given
+    (pages gathered), else from the seeded generator."""
+    ctx = wl.ctx_len[s]
+    nb = (ctx + wl.block_size - 1) // wl.block_size
+    if cache is not None:
+        pages = wl.page_table[s, :nb].long().to(cache.device)
+        t = cache.index_select(0, pages)                      # [nb][H][bs][D]
+        return t.permute(0, 2, 1, 3).reshape(nb * wl.block_size, t.shape[1], t.shape[3])[:ctx].float().cpu().numpy()
+    return gen.token_tensor(wl, tid, s, torch.arange(ctx), device=dev).float().cpu().numpy()
+
+
+class OracleLeg:
+    """The plain C++ oracle (indexer over every visible block, top-k, sparse attention; double
+    arithmetic, std::thread over independent outputs) timed on the host cores on bounded samples
+    of the step's workloads; the step's oracle time is extrapolated from each workload's time per
+    query row.  Inputs come from the device caches of the timed step when there are any, else
+    from the seeded generator (on the GPU when there is one); preparing them is not timed."""
+
+    def __init__(self, parts=None):
+        from oracle import cpp as C
+        self.C = C
+        C.build()
+        self.parts = parts or []
+        self.dev = "cuda" if torch.cuda.is_available() else "cpu"
+        self.chunks = configs.chunked_prefill_128k()
+        self._prefill_keys = None
+        self._decode = {}
+        self.rng = np.random.default_rng(0)
+        self.report = {"rows": 0, "near_ties": 0, "selection_mismatches": 0, "attn_rows_compared": 0,
+                       "attn_max_abs": 0.0, "attn_sum_abs": 0.0, "attn_elems": 0}
+
+    def _part(self, name):
+        return next((p for p in self.parts if p.name == name), None)
+
+    # ---- prefill: rows drawn uniformly from the 131,072-token chunked prefill
+    def prefill_rows(self, n):
+        full = self.chunks[-1]
+        if self._prefill_keys is None:
+            p0 = self._part("prefill128k/c0")
+            cc = p0.caches if p0 is not None else None
+            self._prefill_keys = {
+                "idx_k": _seq_tokens(full, gen.TID_IDX_K, 0, cc["idx_k"] if cc else None, self.dev),
+                "k": _seq_tokens(full, gen.TID_K, 0, cc["k"] if cc else None, self.dev),
+                "v": _seq_tokens(full, gen.TID_V, 0, cc["v"] if cc else None, self.dev)}
+        gpos = np.sort(self.rng.integers(0, full.ctx_len[0], size=n))
+        q, iq = [], []
+        for g in gpos:
+            c, r = int(g) // 16384, int(g) % 16384
+            wl = self.chunks[c]
+            q.append(gen.token_tensor(wl, gen.TID_Q, 0, torch.tensor([int(g)]), device=self.dev).float().cpu())
+            iq.append(gen.token_tensor(wl, gen.TID_IDX_Q, 0, torch.tensor([int(g)]), device=self.dev).float().cpu())
+        q = torch.cat(q).numpy()
+        iq = torch.cat(iq).numpy()
+        hk = self._prefill_keys
         t0 = time.perf_counter()
-        O.msa_rows(q_all[r:r + 1].float().numpy(), iq_all[r:r + 1].float().numpy(), host["k"], host["v"],
-                   host["idx_k"], pos, wl.num_kv_heads, wl.block_size, wl.topk, wl.max_blocks)
-        t_oracle += time.perf_counter() - t0
-        done += 1
-        if t_oracle > seconds_target or (max_rows and done >= max_rows):
-            break
-    return {"value": done / t_oracle, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
-            "sample": f"{done} query rows drawn uniformly from the 131072-token prefill (indexer over every "
-                      f"visible block, top-k, sparse attention; float64 numpy), {t_oracle:.1f} s of oracle time"}
+        s64, sel, out, lse = self.C.msa_rows(q, iq, hk["k"], hk["v"], hk["idx_k"], gpos, full.num_kv_heads,
+                                             full.block_size, full.topk, full.max_blocks)
+        dt = time.perf_counter() - t0
+        if self.parts:
+            for i, g in enumerate(gpos):
+                p = self._part(f"prefill128k/c{int(g) // 16384}")
+                if p is not None:
+                    self._compare(p, int(g) % 16384, s64[i:i + 1], sel[i:i + 1], out[i:i + 1], np.array([g]))
+        return dt
+
+    # ---- decode: whole sequences of the decode workloads (one query row each)
+    def decode_seq(self, name, s):
+        wl = configs.ALL[name]()
+        p = self._part(name)
+        cc = p.caches if p is not None else None
+        key = (name, s)
+        if key not in self._decode:
+            if len(self._decode) > 2:
+                self._decode.clear()
+            self._decode[key] = _seq_tokens(wl, gen.TID_IDX_K, s, cc["idx_k"] if cc else None, self.dev)
+        ik = self._decode[key]
+        nb = (wl.ctx_len[s] + wl.block_size - 1) // wl.block_size
+        if cc is not None:
+            k, v = _Blocks(cc["k"], wl.page_table[s, :nb]), _Blocks(cc["v"], wl.page_table[s, :nb])
+        else:
+            k = gen.token_tensor(wl, gen.TID_K, s, torch.arange(wl.ctx_len[s]), device=self.dev).float().cpu().numpy()
+            v = gen.token_tensor(wl, gen.TID_V, s, torch.arange(wl.ctx_len[s]), device=self.dev).float().cpu().numpy()
+        rows = list(range(wl.q_start[s], wl.q_start[s + 1]))
+        pos = wl.positions()[rows].numpy()
+        q = gen.query_rows(wl, gen.TID_Q, device=self.dev)[rows].float().cpu().numpy() if p is None else \
+            p.q[rows].float().cpu().numpy()
+        iq = gen.query_rows(wl, gen.TID_IDX_Q, device=self.dev)[rows].float().cpu().numpy() if p is None else \
+            p.idx_q[rows].float().cpu().numpy()
+        t0 = time.perf_counter()
+        s64, sel, out, lse = self.C.msa_rows(q, iq, k, v, ik, pos, wl.num_kv_heads, wl.block_size, wl.topk,
+                                             wl.max_blocks)
+        dt = time.perf_counter() - t0
+        if p is not None:
+            for i, r in enumerate(rows):
+                self._compare(p, r, s64[i:i + 1], sel[i:i + 1], out[i:i + 1], pos[i:i + 1])
+        return dt, len(rows)
+
+    def _compare(self, p, r, s64, sel, out, pos):
+        """Parity of the step's own results on a sampled row: selection (exact outside near-ties),
+        and the attention output where the selections agree."""
+        near, _, _ = self.C.boundary_gap(s64, pos, p.wl.topk, p.wl.block_size)
+        got_sel = p.sel[r].cpu().numpy()
+        rep = self.report
+        rep["rows"] += 1
+        rep["near_ties"] += int(near.sum())
+        same = np.array_equal(got_sel, sel[0])
+        if not same:
+            rep["selection_mismatches"] += 1
+            return
+        err = np.abs(p.out[r].float().cpu().numpy().astype(np.float64) - out[0])
+        rep["attn_rows_compared"] += 1
+        rep["attn_max_abs"] = max(rep["attn_max_abs"], float(err.max()))
+        rep["attn_sum_abs"] += float(err.sum())
+        rep["attn_elems"] += int(err.size)
+
+    def run(self, seconds=20.0):
+        """Oracle time per query row of each workload of the default step, then the extrapolated
+        step.  Budget: about half the seconds on prefill rows, the rest on decode sequences."""
+        per_row, used, n_rows = {}, {}, {}
+        # prefill rows in batches until the budget is spent
+        t_pre, n_pre, batch = 0.0, 0, 16
+        while t_pre < 0.5 * seconds:
+            t_pre += self.prefill_rows(batch)
+            n_pre += batch
+            batch = min(256, batch * 2)
+        per_row["prefill_128k"] = t_pre / n_pre
+        used["prefill_128k"], n_rows["prefill_128k"] = t_pre, n_pre
+        for name, share in (("decode_128k", 0.3), ("decode_1m", 0.2)):
+            wl_n = configs.ALL[name]().num_seqs
+            t, n, s = 0.0, 0, 0
+            while (t < share * seconds or n == 0) and s < wl_n:
+                dt, k = self.decode_seq(name, int(self.rng.integers(0, wl_n)))
+                t, n, s = t + dt, n + k, s + 1
+            per_row[name] = t / n
+            used[name], n_rows[name] = t, n
+        tokens = {"prefill_128k": 131072, "decode_128k": 64, "decode_1m": 8}
+        step_s = sum(tokens[k] * per_row[k] for k in tokens)
+        rep = dict(self.report)
+        if rep["attn_elems"]:
+            rep["attn_mean_abs"] = rep["attn_sum_abs"] / rep["attn_elems"]
+        rep.pop("attn_sum_abs")
+        rep.pop("attn_elems")
+        sample = ("C++ oracle (double; std::thread over independent outputs) on "
+                  + ", ".join(f"{n_rows[k]} {k} rows ({used[k]:.1f} s)" for k in per_row)
+                  + "; the step's time extrapolated from each workload's time per row"
+                  + " (131072 prefill + 64 + 8 decode rows)")
+        return {"value": sum(tokens.values()) / step_s, "unit": "tokens/s", "cores": int(self.C.threads()),
+                "cpu_model": cpu_model(), "kind": "oracle", "sample": sample,
+                "seconds_per_row": per_row, "extrapolated_step_s": step_s,
+                "parity": rep if self.parts else None}
 
 
 # ------------------------------------------------------------------ main
@@ -436,17 +569,19 @@ def barrier(ws):
 
 
 def run_reference(args, rank, ws):
+    """The oracle as it stands, timed on the host cores: each step a bounded sample of the step's
+    workloads (no GPU kernel of this repository runs)."""
     if rank != 0:
         return
-    steps = []
+    leg = OracleLeg()
     for _ in range(args.warmup):
-        oracle_sample(seconds_target=2.0, max_rows=4)
-    for _ in range(args.steps):
-        steps.append(oracle_sample(seconds_target=20.0 / max(1, args.steps)))
+        leg.run(seconds=1.0)
+    steps = [leg.run(seconds=max(4.0, 60.0 / max(1, args.steps))) for _ in range(args.steps)]
     val = statistics.median(s["value"] for s in steps)
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": steps[-1]["extrapolated_step_s"] * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded generator)",
             "config": {"workload": args.workload, "sample": steps[-1]["sample"]},
             "cpu_baseline": dict(steps[-1], value=val),
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -703,7 +838,10 @@ def main():
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample()
+        try:
+            cpu = OracleLeg(parts).run(seconds=20.0) if args.workload == "msa_128k_1m" else None
+        except Exception as exc:  # noqa: BLE001
+            cpu = {"error": str(exc)[:300]}
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import block_sparse_long_13_b200 as msa
-from oracle import msa_oracle as O
+from oracle import cpp as O   # the plain C++ oracle (pinned, and checked against the numpy one)
 from workloads import configs, gen
 
 from . import harness as H

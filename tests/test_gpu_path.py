@@ -30,7 +30,7 @@ def _check_chain(d, rows_by_seq, path, report):
     for s, rows in rows_by_seq.items():
         ref64 = H.oracle_scores_rows(d, s, rows)
         worst = max(worst, H.compare_scores(got_s[rows], ref64, pos[rows], wl.block_size))
-        from oracle import msa_oracle as O
+        from oracle import cpp as O
         ref_sel = O.select_blocks(ref64.astype(np.float32), pos[rows], wl.topk, wl.block_size)
         n, m, b = H.compare_selection(got_sel[rows], ref_sel, ref64, pos[rows], wl.topk, wl.block_size)
         tot_near, tot_mism, tot_bad = tot_near + n, tot_mism + m, tot_bad + b

@@ -1,4 +1,4 @@
-"""Pins of the CPU oracle against things other than itself.
+"""Pins of the CPU oracles (float64 numpy and plain C++) against things other than themselves.
 
 * hand-worked fixtures under tests/golden/ (each cites the page rule it follows);
 * brute force with pure-Python loops on tiny integer inputs (exact in float64);
@@ -15,9 +15,16 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import msa_oracle as O
+from oracle import cpp as oracle_cpp
+from oracle import msa_oracle as oracle_numpy
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(params=["numpy", "cpp"])
+def O(request):
+    """Every pin runs against both oracles: the float64 numpy one and the plain C++ one."""
+    return oracle_numpy if request.param == "numpy" else oracle_cpp
 
 
 def _num(x):
@@ -35,7 +42,7 @@ def _load(name):
 
 # ---------------------------------------------------------------- golden fixtures
 
-def test_golden_scores_handworked():
+def test_golden_scores_handworked(O):
     g = _load("scores_handworked.json")
     k = np.array(g["idx_k"], dtype=np.float64)
     q = np.array(g["idx_q"], dtype=np.float64)
@@ -45,7 +52,7 @@ def test_golden_scores_handworked():
     np.testing.assert_array_equal(s2, np.array(_num(g["expected_two_groups"])))
 
 
-def test_golden_topk_handworked():
+def test_golden_topk_handworked(O):
     g = _load("topk_handworked.json")
     for c in g["cases"]:
         s = np.array(_num(c["scores"]), dtype=np.float32)[None, None, :]
@@ -53,7 +60,7 @@ def test_golden_topk_handworked():
         assert got[0, 0].tolist() == c["expected"], c
 
 
-def test_golden_attention_handworked():
+def test_golden_attention_handworked(O):
     g = _load("attention_handworked.json")
     k = np.array(g["k"], dtype=np.float64)
     v = np.array(g["v"], dtype=np.float64)
@@ -100,7 +107,7 @@ def _brute_scores(q, k, pos, Hkv, blk, nb):
 
 
 @pytest.mark.parametrize("Hi,Hkv", [(4, 2), (4, 1), (2, 2)])
-def test_scores_brute_force_tiny(Hi, Hkv):
+def test_scores_brute_force_tiny(O, Hi, Hkv):
     rng = np.random.default_rng(1)
     L, blk, di, n = 37, 8, 5, 9
     k = rng.integers(-4, 5, size=(L, Hi, di)).astype(np.float64)
@@ -112,7 +119,7 @@ def test_scores_brute_force_tiny(Hi, Hkv):
     np.testing.assert_array_equal(got, want)   # integer data: exact in float64
 
 
-def test_scores_closed_form_constant_block():
+def test_scores_closed_form_constant_block(O):
     rng = np.random.default_rng(2)
     L, blk, Hi, di = 64, 16, 4, 8
     k = rng.standard_normal((L, Hi, di))
@@ -126,7 +133,7 @@ def test_scores_closed_form_constant_block():
             assert abs(s[r, g, 1] - want) < 1e-12
 
 
-def test_scores_single_dominant_key_and_causality():
+def test_scores_single_dominant_key_and_causality(O):
     rng = np.random.default_rng(3)
     L, blk, Hi, di = 96, 32, 2, 4
     k = rng.standard_normal((L, Hi, di)) * 0.01
@@ -146,7 +153,7 @@ def test_scores_single_dominant_key_and_causality():
     assert np.isneginf(s2[0, 0, 1:]).all() and np.isneginf(s2[1, 0, 2])
 
 
-def test_scores_positive_scaling_keeps_selection():
+def test_scores_positive_scaling_keeps_selection(O):
     rng = np.random.default_rng(4)
     L, blk, Hi, di = 512, 16, 4, 8
     k = rng.standard_normal((L, Hi, di))
@@ -173,7 +180,7 @@ def _lexsort_select(row, cur, topk):
     return sel + [-1] * (topk - len(sel))
 
 
-def test_topk_matches_full_stable_sort():
+def test_topk_matches_full_stable_sort(O):
     rng = np.random.default_rng(5)
     n, G, nb, blk = 60, 3, 70, 4
     s = rng.standard_normal((n, G, nb)).astype(np.float32)
@@ -190,7 +197,7 @@ def test_topk_matches_full_stable_sort():
                 assert got[r, g].tolist() == want, (topk, r, g)
 
 
-def test_topk_invariants():
+def test_topk_invariants(O):
     rng = np.random.default_rng(6)
     n, G, nb, blk, topk = 200, 2, 300, 128, 16
     s = rng.standard_normal((n, G, nb)).astype(np.float32)
@@ -215,7 +222,7 @@ def test_topk_invariants():
                         assert s[r, g, b] <= worst
 
 
-def test_near_tie_report():
+def test_near_tie_report(O):
     blk = 1
     s = np.array([[[5.0, 3.0, 3.0005, 1.0, 0.0]], [[5.0, 3.0, 2.0, 1.0, 0.0]]])
     near, a, b = O.boundary_gap(s, [4, 4], 3, blk)   # 2 free slots
@@ -243,7 +250,7 @@ def _sdpa(q, k, v, mask, scale):
 
 
 @pytest.mark.parametrize("L,blk", [(300, 32), (100, 128)])
-def test_attention_all_blocks_is_dense_causal(L, blk):
+def test_attention_all_blocks_is_dense_causal(O, L, blk):
     rng = np.random.default_rng(7)
     Hq, Hkv, d = 8, 2, 16
     q = rng.standard_normal((L, Hq, d))
@@ -262,7 +269,7 @@ def test_attention_all_blocks_is_dense_causal(L, blk):
     np.testing.assert_allclose(lse, wlse, atol=1e-12)
 
 
-def test_attention_subset_is_masked_attention():
+def test_attention_subset_is_masked_attention(O):
     rng = np.random.default_rng(8)
     L, blk, Hq, Hkv, d, topk = 256, 16, 6, 3, 8, 4
     q = rng.standard_normal((L, Hq, d))
@@ -285,7 +292,7 @@ def test_attention_subset_is_masked_attention():
     np.testing.assert_allclose(lse, wlse, atol=1e-12)
 
 
-def test_attention_value_special_cases():
+def test_attention_value_special_cases(O):
     rng = np.random.default_rng(9)
     L, blk, Hq, Hkv, d = 64, 16, 4, 1, 8
     q = rng.standard_normal((L, Hq, d))
@@ -306,7 +313,7 @@ def test_attention_value_special_cases():
         assert abs(out[r, h, 0] - math.exp(logit - lse[r, h])) < 1e-12
 
 
-def test_merge_is_associative():
+def test_merge_is_associative(O):
     rng = np.random.default_rng(10)
     L, blk, Hq, Hkv, d = 160, 16, 4, 2, 8
     q = rng.standard_normal((5, Hq, d))
@@ -337,7 +344,7 @@ def test_merge_is_associative():
 
 # ---------------------------------------------------------------- planted mistakes
 
-def test_fixtures_catch_plausible_slips():
+def test_fixtures_catch_plausible_slips(O):
     """The hand-worked fixtures are sensitive to the slips a restatement could
     make: off-by-one causality, max instead of sum over a group's heads,
     mean instead of max pooling, and ties going to the higher block id."""
