@@ -102,8 +102,8 @@ class Part:
         self.fused = fused and kind == "prefill" and wl.topk <= 16
         self.scores = None if self.fused else torch.empty((T, G, nb), dtype=torch.float32, device=dev)
         # kernels of ours per run: indexer (+ top-k), then attention: prefill = schedule (4 kernels),
-        # block-major attention, merge; decode = one kernel
-        self.launches = (1 if self.fused else 2) + (6 if kind == "prefill" else 1)
+        # block-major attention, merge; decode = work-item plan + attention
+        self.launches = (1 if self.fused else 2) + (6 if kind == "prefill" else 2)
         self.pos = wl.positions()
 
     def run(self, ws, ev=None, stream=None, stop_after="attn"):
@@ -303,6 +303,45 @@ def time_next_rows(parts, pk):
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"qk_rope_insert_kernel": {"part": p.name, "rows": T, "ms_per_call": ms, "bytes_per_call": nbytes,
                                       "gbs": gbs, "frac": gbs / pk["hbm_gbs"], "status": int(msa.device_status())}}
+
+
+def time_fp8_indexer(parts, pk):
+    """The streaming indexer over an e4m3 copy of a decode workload's indexer keys (the FP8 cache
+    path), timed by itself: the codes are written once with one scale (torch, untimed), then 20
+    calls after 3 warm-ups, CUDA events.  Algorithmic bytes: every visible key's 64 codes per
+    indexer head (half the bf16 bytes)."""
+    import block_sparse_long_13_b200 as msa
+    p = next((x for x in parts if x.name == "decode_128k"), None) or next(
+        (x for x in parts if x.kind == "decode"), None)
+    if p is None:
+        return None
+    k = p.caches["idx_k"]
+    s = float(k.float().abs().max()) / 448.0
+    codes = torch.empty(k.shape, dtype=torch.uint8, device="cuda")
+    for i in range(0, k.shape[0], 4096):       # written in slices to bound the temporaries
+        codes[i:i + 4096] = torch.clamp(k[i:i + 4096].float() / s, -448.0, 448.0).to(
+            torch.float8_e4m3fn).view(torch.uint8)
+    scores = torch.empty_like(p.scores)
+
+    def call():
+        msa.index_scores_fp8(p.cfg, p.batch, p.idx_q, codes, s, scores)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 20
+    e0.record()
+    for _ in range(n):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    wl = p.wl
+    nbytes = float(sum(wl.ctx_len)) * wl.idx_heads * wl.idx_dim
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del codes
+    return {"part": p.name, "ms_per_call": ms, "bytes_per_call": nbytes, "gbs": gbs,
+            "frac": gbs / pk["hbm_gbs"], "frac_8tbs": gbs / pk["hbm_gbs_spec"], "status": int(msa.device_status())}
 
 
 # ------------------------------------------------------------------ clocks
@@ -824,6 +863,12 @@ def main():
             next_rows = time_next_rows(parts, pk)
         except Exception as exc:  # noqa: BLE001
             next_rows = {"error": str(exc)[:200]}
+        try:
+            fp8 = time_fp8_indexer(parts, pk)
+            if fp8 is not None:
+                next_rows = dict(next_rows or {}, index_decode_kernel_e4m3=fp8)
+        except Exception as exc:  # noqa: BLE001
+            next_rows = dict(next_rows or {}, index_decode_kernel_e4m3={"error": str(exc)[:200]})
 
     # the other workloads of the parity set, timed on their own after the step (not in `value`)
     if rank == 0 and args.workload == "msa_128k_1m" and not args.no_extra:

@@ -28,7 +28,7 @@ EXPORTS = (
     "msa_prefill_workspace_bytes", "msa_decode_workspace_bytes", "msa_get_device_status",
     "msa_set_wait_limit_ns", "msa_debug_wait_timeout", "msa_status_string", "msa_last_error",
     "msa_version", "msa_attn_decode_noalloc", "msa_index_topk", "msa_set_timing_events",
-    "msa_qknorm_rope_insert", "msa_merge_partials",
+    "msa_qknorm_rope_insert", "msa_merge_partials", "msa_index_scores_fp8",
 )
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_CUDA, MSA_ERR_TIMEOUT, MSA_ERR_DEVICE_BOUNDS = range(6)
@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     cfgp, batp = ctypes.POINTER(_CConfig), ctypes.POINTER(_CBatch)
     sigs = {
         "msa_index_scores": [cfgp, batp, P, P, P, P],
+        "msa_index_scores_fp8": [cfgp, batp, P, P, ctypes.c_float, P, P],
         "msa_topk_blocks": [cfgp, batp, P, P, P],
         "msa_index_topk": [cfgp, batp, P, P, P, P],
         "msa_set_timing_events": [P, ctypes.c_int32],
@@ -182,6 +183,17 @@ def index_scores(cfg: Config, batch: Batch, idx_q, idx_k_cache, block_scores, st
                                 _need(idx_q, torch.bfloat16, "idx_q"),
                                 _need(idx_k_cache, torch.bfloat16, "idx_k_cache"),
                                 _need(block_scores, torch.float32, "block_scores"), _stream(stream)))
+
+
+def index_scores_fp8(cfg: Config, batch: Batch, idx_q, idx_k_cache_e4m3, k_scale: float, block_scores,
+                     stream=None) -> None:
+    """Indexer block scores over an e4m3 indexer-key cache (uint8 codes, value = code * k_scale);
+    decode and verify calls (at most 8 queries per sequence)."""
+    lib = load_library()
+    _check(lib.msa_index_scores_fp8(ctypes.byref(cfg._c()), ctypes.byref(batch._c()),
+                                    _need(idx_q, torch.bfloat16, "idx_q"),
+                                    _need(idx_k_cache_e4m3, torch.uint8, "idx_k_cache_e4m3"), float(k_scale),
+                                    _need(block_scores, torch.float32, "block_scores"), _stream(stream)))
 
 
 def topk_blocks(cfg: Config, batch: Batch, block_scores, block_idx, stream=None) -> None:

@@ -15,12 +15,14 @@
 // concatenation").  K_b and V_b (128 x 128 bf16 each, one TMA load per
 // bucket per CTA) stay in shared memory while the CTA walks consecutive
 // tiles of the same bucket.  S = Q K^T and O = P V run on tcgen05 with fp32
-// accumulators in TMEM; a 4-warp softmax group reads S rows from TMEM (thread
-// = row), masks keys after the query position (only the query's own block
-// has any), writes P as bf16 back into TMEM, from where the P V MMA reads
-// it (operand A in TMEM: shared-memory bandwidth is left to the S = Q K^T
-// operands and the V tile), and later stores O / l (bf16) and lse = m + ln l
-// as the partial of (t, head, slot).
+// accumulators in TMEM; two 4-warp softmax groups take alternate tiles, each
+// with its own S, P and O in TMEM: thread = row reads its S row, masks keys
+// after the query position (only the query's own block has any), writes P as
+// bf16 over the first half of its S columns, from where the P V MMA reads it
+// (operand A in TMEM: shared-memory bandwidth is left to the S = Q K^T
+// operands and the V tile), and later reads its own O accumulator and stores
+// O / l (bf16) and lse = m + ln l as the partial of (t, head, slot).  With an
+// O per group, one group's epilogue never holds up the other group's P V.
 //
 // Phase 2 (merge): out(t, h) = sum_slots exp(lse_s - L) O_s with
 // L = log sum_s exp(lse_s); lse(t, h) = L.
@@ -226,8 +228,9 @@ struct AttnPrefillArgs {
 constexpr int ATTP_QBUF = 3;      // gathered query tiles in flight (the gather latency needs > 2)
 constexpr int ATTP_QBYTES = 32768, ATTP_KVBYTES = 32768, ATTP_STAGE = 32768;
 constexpr int ATTP_SMEM = ATTP_QBUF * ATTP_QBYTES + 2 * ATTP_KVBYTES + 2 * ATTP_STAGE + 1024;
-// TMEM columns: S[2] (fp32) at 0 / 128, P[2] (bf16 pairs) at 256 / 320, O (fp32) at 384
-constexpr uint32_t ATTP_TM_S = 0, ATTP_TM_P = 256, ATTP_TM_O = 384;
+// TMEM columns: S[w] (fp32) at 0 / 128, P[w] (bf16 pairs) over the first 64 columns of S[w], O[w] (fp32)
+// at 256 / 384; w = the softmax warpgroup = the tile's parity
+constexpr uint32_t ATTP_TM_S = 0, ATTP_TM_O = 256;
 
 __global__ void __launch_bounds__(ATTP_THREADS, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [total_q*Hq][128]
@@ -243,10 +246,10 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
   uint8_t* o_s = v_s + ATTP_KVBYTES;                    // 2 x 32 KiB: [half][128 rows][64 dims]
 
   // Per warpgroup w (its own tile sequence, so a parity never runs two phases ahead): s_full[w] S is in
-  // TMEM, p_full[w] P is in TMEM (one arrival per warp), o_full[w] the O accumulator holds its tile.
-  // o_empty: O has been read (one arrival per warp); only the UMMA thread waits on it, in tile order.
+  // TMEM, p_full[w] P is in TMEM (one arrival per warp), o_full[w] O[w] holds its tile, o_empty[w] O[w]
+  // has been read (one arrival per warp).
   __shared__ uint64_t kv_full, kv_empty, q_full[ATTP_QBUF], q_empty[ATTP_QBUF], s_full[2], p_full[2], o_full[2],
-      o_empty, drain_bar;
+      o_empty[2], drain_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
 
@@ -263,8 +266,8 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
       mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 4);
     }
-    mbar_init(&o_empty, 4);
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
   }
@@ -395,9 +398,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ UMMA issuer
-    // Tile i: S(i) = Q K^T into S[i % 2] (A and B from shared memory), then O = P(i-1) V with
-    // P(i-1) read from TMEM.  tcgen05.commit tracks every earlier MMA of this thread, so the
-    // s_full(i) signal also means PV(i-2) has finished reading P[i % 2].
+    // Tile i: S(i) = Q K^T into S[i % 2] (A and B from shared memory), then O[(i-1) % 2] = P(i-1) V with
+    // P(i-1) read from TMEM over the first half of S[(i-1) % 2].  S(i) overwrites the columns P V(i-2)
+    // read: this thread issued P V(i-2) first, and its MMAs run in issue order.
     // This one thread's instruction latency is on the critical path: descriptors are built once
     // (only the 14-bit start address, in 16-byte units, moves) and ring positions are counters.
     const uint32_t id_s = idesc_bf16(128, 128, false, false);
@@ -410,14 +413,16 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
     int cur_bucket = -1;
     uint32_t kvit = 0;
     bool pv_pending = false;
-    auto issue_pv = [&](int j) -> bool {  // O = P[j%2] V
+    auto issue_pv = [&](int j) -> bool {  // O[j%2] = P[j%2] V
       const int pb = j & 1;
-      if (!mbar_wait(&p_full[pb], (j >> 1) & 1, &s_abort)) return false;
-      if (!mbar_wait(&o_empty, (j & 1) ^ 1, &s_abort)) return false;   // tile j-1's O has been read
+      const uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
+      if (!mbar_wait(&p_full[pb], ph, &s_abort)) return false;
+      if (!mbar_wait(&o_empty[pb], ph ^ 1u, &s_abort)) return false;   // tile j-2's O has been read
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)   // 16 keys per step: 2048 bytes of V rows
-        umma_bf16_ts(tmem + ATTP_TM_O, tmem + ATTP_TM_P + pb * 64 + kk * 8, vdesc0 + 128 * kk, id_pv, kk > 0 ? 1u : 0u);
+        umma_bf16_ts(tmem + ATTP_TM_O + pb * 128, tmem + ATTP_TM_S + pb * 128 + kk * 8, vdesc0 + 128 * kk, id_pv,
+                     kk > 0 ? 1u : 0u);
       umma_commit(&o_full[pb]);
       return true;
     };
@@ -536,7 +541,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
           if (q2 & 1) l1 += p0 + p1; else l0 += p0 + p1;
           pk[q2] = pack_bf16(p0, p1);
         }
-        tmem_st32(lane_addr + ATTP_TM_P + w * 64 + half * 32, pk);
+        tmem_st32(lane_addr + ATTP_TM_S + w * 128 + half * 32, pk);   // S columns already in registers
       }
       tmem_st_wait();
       tc_fence_before();
@@ -548,14 +553,15 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,     // q as [tot
       if (!mbar_wait_warp(&o_full[w], static_cast<uint32_t>(j & 1), &s_abort)) break;
       tc_fence_after();
       float o0[32], o1[32], o2[32], o3[32];
-      tmem_ld32(lane_addr + ATTP_TM_O, o0);
-      tmem_ld32(lane_addr + ATTP_TM_O + 32, o1);
-      tmem_ld32(lane_addr + ATTP_TM_O + 64, o2);
-      tmem_ld32(lane_addr + ATTP_TM_O + 96, o3);
+      const uint32_t o_addr = lane_addr + ATTP_TM_O + w * 128;
+      tmem_ld32(o_addr, o0);
+      tmem_ld32(o_addr + 32, o1);
+      tmem_ld32(o_addr + 64, o2);
+      tmem_ld32(o_addr + 96, o3);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty);
+      if (lane == 0) mbar_arrive(&o_empty[w]);
       if (lane == 0) bulk_wait_read_all();        // this warp's previous stores have left its staging rows
       __syncwarp();
       const float inv = 1.f / l;

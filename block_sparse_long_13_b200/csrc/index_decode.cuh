@@ -22,6 +22,8 @@
 // memory; the block max is a warp redux.sync on order-preserving integer
 // keys, then a per-group sum over the heads.
 #pragma once
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace msa {
@@ -44,10 +46,29 @@ struct IdxDecodeArgs {
   const int32_t* page_table;    // [num_seqs][max_blocks]
   int num_seqs, max_blocks, num_pages, Hi, Hkv, hg, block_size;
   int stage_bytes, stages;
+  float k_scale;                // e4m3 keys: value = code * k_scale (1 for bf16 keys)
 };
 
-// NQ: compile-time bound on the queries of any sequence (1, 2, 4 or 8)
-template <int NQ>
+// 16 e4m3 codes (one 16-byte chunk of a key row) widened exactly to fp32: pairs through the
+// packed e4m3x2 -> f16x2 conversion, then f16 -> f32 (both exact: every e4m3 value is an f16 value).
+__device__ __forceinline__ void e4m3x16_to_f32(const uint4 w, float (&f)[16]) {
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t lo, hi;
+    const uint16_t b01 = static_cast<uint16_t>(words[i] & 0xFFFFu), b23 = static_cast<uint16_t>(words[i] >> 16);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(lo) : "h"(b01));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hi) : "h"(b23));
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+    f[4 * i + 0] = a.x; f[4 * i + 1] = a.y; f[4 * i + 2] = b.x; f[4 * i + 3] = b.y;
+  }
+}
+
+// NQ: compile-time bound on the queries of any sequence (1, 2, 4 or 8).  E4M3: the indexer keys are
+// e4m3 codes (64-byte rows, 64-byte TMA swizzle) read back as code * k_scale; else bf16 (128-byte rows,
+// 128-byte swizzle).
+template <int NQ, bool E4M3 = false>
 __global__ void __launch_bounds__(idxd_threads(NQ), 1)
 index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeArgs a) {
   constexpr int NG = idxd_groups(NQ);
@@ -159,7 +180,8 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
         float tot = 0.f;
         for (int hl = 0; hl < a.hg; ++hl) {
           const uint32_t* pp = s_part[grp][pbuf][cl][hl];
-          tot += key_to_float(max(max(pp[0], pp[1]), max(pp[2], pp[3])));
+          const float mx = key_to_float(max(max(pp[0], pp[1]), max(pp[2], pp[3])));
+          tot += E4M3 ? mx * a.k_scale : mx;    // max_j q . (c_j s) = s max_j q . c_j for s > 0
         }
         a.scores[(static_cast<long>(pv_row0 + cl) * a.Hkv + pv_g) * a.max_blocks + pv_b] = tot;
       }
@@ -193,27 +215,45 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
       const int j = b * a.block_size + token;  // absolute key position
       const int pbuf = m & 1;
       for (int hl = hl0; hl < a.hg; hl += 2) {
-        // this thread's key row: 64 bf16, 128-byte swizzled
-        const uint8_t* rowp = tile + (hl * 128 + token) * 128;
         float ac0[NQ], ac1[NQ];
 #pragma unroll
         for (int i = 0; i < NQ; ++i) { ac0[i] = 0.f; ac1[i] = 0.f; }
         const int h = g * a.hg + hl;
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((cc ^ (token & 7)) << 4));
-          const float kf[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
-                               bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+        auto dot8 = [&](const float (&kf)[8], int c0) {      // keys c0 .. c0+7 of the row against the queries
 #pragma unroll
           for (int i = 0; i < NQ; ++i) {
             if (NQ == 1 || i < nq) {
-              const float4* qp = reinterpret_cast<const float4*>(s_q + (i * a.Hi + h) * 64 + cc * 8);
+              const float4* qp = reinterpret_cast<const float4*>(s_q + (i * a.Hi + h) * 64 + c0);
               const float4 q0 = qp[0], q1 = qp[1];
               float t0 = ac0[i], t1 = ac1[i];
               t0 = fmaf(q0.x, kf[0], t0); t1 = fmaf(q0.y, kf[1], t1); t0 = fmaf(q0.z, kf[2], t0); t1 = fmaf(q0.w, kf[3], t1);
               t0 = fmaf(q1.x, kf[4], t0); t1 = fmaf(q1.y, kf[5], t1); t0 = fmaf(q1.z, kf[6], t0); t1 = fmaf(q1.w, kf[7], t1);
               ac0[i] = t0; ac1[i] = t1;
             }
+          }
+        };
+        if constexpr (E4M3) {
+          // this thread's key row: 64 e4m3 codes, 64-byte swizzled (16-byte chunk c of row r at c ^ ((r >> 1) & 3))
+          const uint8_t* rowp = tile + (hl * 128 + token) * 64;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((cc ^ ((token >> 1) & 3)) << 4));
+            float kf16[16];
+            e4m3x16_to_f32(w, kf16);
+            const float (&k0)[8] = *reinterpret_cast<const float(*)[8]>(kf16);
+            const float (&k1)[8] = *reinterpret_cast<const float(*)[8]>(kf16 + 8);
+            dot8(k0, cc * 16);
+            dot8(k1, cc * 16 + 8);
+          }
+        } else {
+          // this thread's key row: 64 bf16, 128-byte swizzled
+          const uint8_t* rowp = tile + (hl * 128 + token) * 128;
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((cc ^ (token & 7)) << 4));
+            const float kf[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
+                                 bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+            dot8(kf, cc * 8);
           }
         }
 #pragma unroll

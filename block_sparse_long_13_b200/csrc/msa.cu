@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -14,6 +15,7 @@
 #include "attn_prefill.cuh"
 #include "common.cuh"
 #include "index_decode.cuh"
+#include "index_decode_tc.cuh"
 #include "index_prefill.cuh"
 #include "merge_partials.cuh"
 #include "qk_rope_insert.cuh"
@@ -112,9 +114,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle
+// tensor of `rank` dims (innermost first): bf16 with the 128-byte swizzle by default
 msa_status_t make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
-                      const uint32_t* box) {
+                      const uint32_t* box, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t gd[5], gs[4];
@@ -125,9 +128,8 @@ msa_status_t make_map(CUtensorMap* m, const void* base, int rank, const uint64_t
     es[i] = 1;
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, dtype, rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return MSA_OK;
 }
@@ -171,17 +173,21 @@ PrefillWs prefill_plan(const msa_config_t* c, const msa_batch_t* b) {
   return w;
 }
 
+// Splits per (row, group) of the decode attention: a split holds at most msa::ATTD_MAXB selected
+// slots, and there should be about 2 work items per SM (more items share out more evenly, fewer
+// pay less per-item latency and merge traffic).
 int decode_splits(const msa_config_t* c, const msa_batch_t* b) {
   const long units = static_cast<long>(b->total_q) * c->num_kv_heads;
-  if (units <= 0) return 1;
-  long want = (4L * 148 + units - 1) / units;  // aim at ~4 CTAs per SM of a 148-SM B200
-  if (want < 1) want = 1;
-  if (want > c->topk) want = c->topk;
+  const long min_split = (c->topk + msa::ATTD_MAXB - 1) / msa::ATTD_MAXB;
+  if (units <= 0) return static_cast<int>(min_split);
+  long want = (2L * 148 + units - 1) / units;
+  want = std::max(want, min_split);
+  want = std::min<long>(want, c->topk);
   return static_cast<int>(want);
 }
 
 struct DecodeWs {
-  size_t counters, part_lse, part_o, bytes;
+  size_t part_lse, part_o, items, bytes;
   int nsplit;
 };
 
@@ -191,9 +197,9 @@ DecodeWs decode_plan(const msa_config_t* c, const msa_batch_t* b) {
   const size_t units = static_cast<size_t>(b->total_q) * c->num_kv_heads;
   size_t o = 0;
   auto take = [&](size_t n) { size_t at = o; o = align_up(o + n, 256); return at; };
-  w.counters = take(units * 4);
   w.part_lse = take(units * w.nsplit * 16 * 4);
   w.part_o = take(units * w.nsplit * 16 * 128 * 4);
+  w.items = take(units * w.nsplit * 6 * 16);          // one 96-byte record per work item
   w.bytes = o;
   return w;
 }
@@ -289,6 +295,84 @@ size_t msa_decode_workspace_bytes(const msa_config_t* cfg, const msa_batch_t* ba
   return decode_plan(cfg, batch).bytes;
 }
 
+}  // extern "C"
+
+// The streaming (few queries per sequence) indexer over bf16 or e4m3 keys.
+template <bool E4M3>
+msa_status_t launch_index_decode(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
+                                 const void* idx_k_cache, float k_scale, float* block_scores, cudaStream_t stream) {
+  msa_status_t st;
+  const int Hi = cfg->idx_heads, Hkv = cfg->num_kv_heads, hg = Hi / Hkv;
+  const int esz = E4M3 ? 1 : 2;
+  CUtensorMap tk;
+  {
+    const uint64_t row = 64ull * esz;
+    const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
+    const uint64_t strides[3] = {row, row * 128, static_cast<uint64_t>(Hi) * row * 128};
+    const uint32_t box[4] = {64, 128, static_cast<uint32_t>(hg), 1};
+    if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box,
+                       E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                       E4M3 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+      return st;
+  }
+  const int sms = num_sms();
+  CHECK_SUP(batch->num_seqs <= msa::IDXD_MAXSEQ, "at most %d sequences per streaming indexer call",
+            msa::IDXD_MAXSEQ);
+  msa::IdxDecodeArgs a{};
+  a.idx_q = static_cast<const __nv_bfloat16*>(idx_q);
+  a.scores = block_scores;
+  a.q_start = batch->q_start;
+  a.ctx_len = batch->ctx_len;
+  a.page_table = batch->page_table;
+  a.num_seqs = batch->num_seqs;
+  a.max_blocks = batch->max_blocks_per_seq;
+  a.num_pages = batch->num_pages;
+  a.Hi = Hi;
+  a.Hkv = Hkv;
+  a.hg = hg;
+  a.block_size = cfg->block_size;
+  a.stage_bytes = hg * 128 * 64 * esz;
+  a.k_scale = k_scale;
+  const int mq = batch->max_q_per_seq;
+  if (!E4M3 && mq > 2) {
+    // several queries per sequence: the tensor-core form (its shared-memory traffic does not grow with them)
+    CUtensorMap tq;
+    {
+      const uint64_t dims[3] = {64, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->total_q)};
+      const uint64_t strides[2] = {128, static_cast<uint64_t>(Hi) * 128};
+      const uint32_t box[3] = {64, 1, 16};
+      if ((st = make_map(&tq, idx_q, 3, dims, strides, box)) != MSA_OK) return st;
+    }
+    const int q_tiles = 2 * Hi * msa::IDXT_QHEAD;
+    a.stages = std::min(16, (200 * 1024 - q_tiles) / a.stage_bytes);
+    CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
+    const int smem = a.stages * a.stage_bytes + q_tiles + 1024;
+    auto go_tc = [&](auto kernel) -> msa_status_t {
+      CUDA_TRY(set_smem(kernel, smem));
+      kernel<<<sms, msa::IDXT_THREADS, smem, stream>>>(tk, tq, a);
+      return launched();
+    };
+    if (mq <= 4) return go_tc(msa::index_decode_tc_kernel<4>);
+    return go_tc(msa::index_decode_tc_kernel<8>);
+  }
+  const int nqb = mq <= 1 ? 1 : mq <= 2 ? 2 : mq <= 4 ? 4 : 8;   // compile-time query bound
+  const int q_bytes = msa::idxd_groups(nqb) * nqb * Hi * 64 * 4;   // each consumer group's queries
+  a.stages = std::min(16, (msa::IDXD_SMEM_BUDGET - q_bytes) / a.stage_bytes);
+  CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
+  const int smem = a.stages * a.stage_bytes + q_bytes + 1024;
+  auto go = [&](auto kernel) -> msa_status_t {
+    CUDA_TRY(set_smem(kernel, smem));
+    kernel<<<sms, msa::idxd_threads(nqb), smem, stream>>>(tk, a);
+    return launched();
+  };
+  if (mq <= 1) return go(msa::index_decode_kernel<1, E4M3>);
+  if (mq <= 2) return go(msa::index_decode_kernel<2, E4M3>);
+  if (mq <= 4) return go(msa::index_decode_kernel<4, E4M3>);
+  return go(msa::index_decode_kernel<8, E4M3>);
+}
+
+extern "C" {
+
 msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
                               const void* idx_k_cache, float* block_scores, cudaStream_t stream) {
   msa_status_t st;
@@ -297,49 +381,25 @@ msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch,
   CHECK_ARG(idx_q && idx_k_cache && block_scores, "idx_q, idx_k_cache and block_scores must not be NULL");
   CHECK_ARG(aligned16(idx_q) && aligned16(idx_k_cache) && aligned16(block_scores), "pointers must be 16-byte aligned");
   if (batch->total_q == 0) return MSA_OK;
-  const int Hi = cfg->idx_heads, Hkv = cfg->num_kv_heads, hg = Hi / Hkv;
-  if (batch->max_q_per_seq <= msa::IDXD_MAXQ) {
-    CUtensorMap tk;
-    {
-      const uint64_t dims[4] = {64, 128, static_cast<uint64_t>(Hi), static_cast<uint64_t>(batch->num_pages)};
-      const uint64_t strides[3] = {128, 128 * 128, static_cast<uint64_t>(Hi) * 128 * 128};
-      const uint32_t box[4] = {64, 128, static_cast<uint32_t>(hg), 1};
-      if ((st = make_map(&tk, idx_k_cache, 4, dims, strides, box)) != MSA_OK) return st;
-    }
-    const int sms = num_sms();
-    CHECK_SUP(batch->num_seqs <= msa::IDXD_MAXSEQ, "at most %d sequences per streaming indexer call",
-              msa::IDXD_MAXSEQ);
-    msa::IdxDecodeArgs a{};
-    a.idx_q = static_cast<const __nv_bfloat16*>(idx_q);
-    a.scores = block_scores;
-    a.q_start = batch->q_start;
-    a.ctx_len = batch->ctx_len;
-    a.page_table = batch->page_table;
-    a.num_seqs = batch->num_seqs;
-    a.max_blocks = batch->max_blocks_per_seq;
-    a.num_pages = batch->num_pages;
-    a.Hi = Hi;
-    a.Hkv = Hkv;
-    a.hg = hg;
-    a.block_size = cfg->block_size;
-    a.stage_bytes = hg * 128 * 64 * 2;
-    const int mq = batch->max_q_per_seq;
-    const int nqb = mq <= 1 ? 1 : mq <= 2 ? 2 : mq <= 4 ? 4 : 8;   // compile-time query bound
-    const int q_bytes = msa::idxd_groups(nqb) * nqb * Hi * 64 * 4;   // each consumer group's queries
-    a.stages = std::min(16, (msa::IDXD_SMEM_BUDGET - q_bytes) / a.stage_bytes);
-    CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
-    const int smem = a.stages * a.stage_bytes + q_bytes + 1024;
-    auto go = [&](auto kernel) -> msa_status_t {
-      CUDA_TRY(set_smem(kernel, smem));
-      kernel<<<sms, msa::idxd_threads(nqb), smem, stream>>>(tk, a);
-      return launched();
-    };
-    if (mq <= 1) return go(msa::index_decode_kernel<1>);
-    if (mq <= 2) return go(msa::index_decode_kernel<2>);
-    if (mq <= 4) return go(msa::index_decode_kernel<4>);
-    return go(msa::index_decode_kernel<8>);
-  }
+  if (batch->max_q_per_seq <= msa::IDXD_MAXQ)
+    return launch_index_decode<false>(cfg, batch, idx_q, idx_k_cache, 1.f, block_scores, stream);
   return launch_index_prefill<false>(cfg, batch, idx_q, idx_k_cache, block_scores, nullptr, stream);
+}
+
+msa_status_t msa_index_scores_fp8(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
+                                  const void* idx_k_cache_e4m3, float k_scale, float* block_scores,
+                                  cudaStream_t stream) {
+  msa_status_t st;
+  if ((st = check_config(cfg)) != MSA_OK) return st;
+  if ((st = check_batch(batch)) != MSA_OK) return st;
+  CHECK_ARG(idx_q && idx_k_cache_e4m3 && block_scores, "idx_q, idx_k_cache_e4m3 and block_scores must not be NULL");
+  CHECK_ARG(aligned16(idx_q) && aligned16(idx_k_cache_e4m3) && aligned16(block_scores),
+            "pointers must be 16-byte aligned");
+  CHECK_ARG(std::isfinite(k_scale) && k_scale > 0.f, "k_scale must be positive and finite");
+  CHECK_SUP(batch->max_q_per_seq <= msa::IDXD_MAXQ, "the e4m3 indexer handles at most %d queries per sequence",
+            msa::IDXD_MAXQ);
+  if (batch->total_q == 0) return MSA_OK;
+  return launch_index_decode<true>(cfg, batch, idx_q, idx_k_cache_e4m3, k_scale, block_scores, stream);
 }
 
 msa_status_t msa_topk_blocks(const msa_config_t* cfg, const msa_batch_t* batch, const float* block_scores,
@@ -504,9 +564,6 @@ msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, 
   if (batch->total_q == 0) return MSA_OK;
   char* ws = static_cast<char*>(workspace);
   msa::AttnDecodeArgs a{};
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
-  a.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
   a.block_idx = block_idx;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse = lse;
@@ -515,7 +572,7 @@ msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, 
   a.page_table = batch->page_table;
   a.part_o = reinterpret_cast<float*>(ws + w.part_o);
   a.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
-  a.counters = reinterpret_cast<int*>(ws + w.counters);
+  a.items = reinterpret_cast<int4*>(ws + w.items);
   a.num_seqs = batch->num_seqs;
   a.total_q = batch->total_q;
   a.Hq = cfg->num_q_heads;
@@ -527,10 +584,34 @@ msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, 
   a.nsplit = w.nsplit;
   a.scale_log2 = softmax_scale(cfg) * 1.4426950408889634f;
   const size_t units = static_cast<size_t>(batch->total_q) * cfg->num_kv_heads;
-  CUDA_TRY(cudaMemsetAsync(a.counters, 0, units * 4, stream));
-  CUDA_TRY(set_smem(msa::attn_decode_kernel, msa::ATTD_SMEM));   // with the static arrays: above the 48 KiB default
-  msa::attn_decode_kernel<<<static_cast<unsigned>(units * w.nsplit), msa::ATTD_THREADS, msa::ATTD_SMEM, stream>>>(a);
-  return launched();
+  CHECK_SUP(units * w.nsplit < (size_t(1) << 31), "too many (row, group, split) work items");
+  a.per = (cfg->topk + w.nsplit - 1) / w.nsplit;
+  a.n_items = static_cast<int>(units * w.nsplit);
+  CUtensorMap tq, tk, tv;
+  {
+    const uint64_t dims[2] = {128, static_cast<uint64_t>(batch->total_q) * cfg->num_q_heads};
+    const uint64_t strides[1] = {256};
+    const uint32_t box[2] = {64, 16};
+    if ((st = make_map(&tq, q, 2, dims, strides, box)) != MSA_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {128, static_cast<uint64_t>(batch->num_pages) * cfg->num_kv_heads * 128};
+    const uint64_t strides[1] = {256};
+    const uint32_t box[2] = {64, 128};
+    if ((st = make_map(&tk, k_cache, 2, dims, strides, box)) != MSA_OK) return st;
+    if ((st = make_map(&tv, v_cache, 2, dims, strides, box)) != MSA_OK) return st;
+  }
+  msa::attn_decode_plan_kernel<<<static_cast<unsigned>((a.n_items + 255) / 256), 256, 0, stream>>>(a);
+  if ((st = launched()) != MSA_OK) return st;
+  CUDA_TRY(set_smem(msa::attn_decode_kernel, msa::ATTD_SMEM));
+  const int grid = static_cast<int>(std::min<long>(a.n_items, num_sms()));
+  msa::attn_decode_kernel<<<grid, msa::ATTD_THREADS, msa::ATTD_SMEM, stream>>>(tq, tk, tv, a);
+  if ((st = launched()) != MSA_OK) return st;
+  if (w.nsplit > 1) {
+    msa::attn_decode_merge_kernel<<<static_cast<unsigned>(units), 256, 0, stream>>>(a);
+    if ((st = launched()) != MSA_OK) return st;
+  }
+  return MSA_OK;
 }
 
 msa_status_t msa_qknorm_rope_insert(const msa_config_t* cfg, const msa_batch_t* batch, void* q, const void* k_new,
@@ -622,7 +703,7 @@ msa_status_t msa_debug_wait_timeout(cudaStream_t stream) {
 // framework that passes it only input and output buffers has no allocator of
 // its own, and a serving loop may forbid cudaMalloc on the per-step path
 // (it can synchronize the device and its latency is unbounded).  For them
-// msa_attn_decode_noalloc keeps the split-K partials and counters of the
+// msa_attn_decode_noalloc keeps the split partials and work-item records of the
 // decode attention in this fixed device array instead.  The array is part of
 // the library's device code: every GPU that loads the library holds it until
 // the process exits.
@@ -670,7 +751,6 @@ extern "C" msa_status_t msa_attn_decode_noalloc(const msa_config_t* cfg, const m
                 need, kNoAllocScratchBytes);
   void* scratch = nullptr;
   if ((st = noalloc_scratch(stream, &scratch)) != MSA_OK) return st;
-  // the decode path clears its counters itself (cudaMemsetAsync, no allocation)
   return msa_attn_decode(cfg, batch, q, k_cache, v_cache, block_idx, out, lse, scratch, kNoAllocScratchBytes,
                          stream);
 }

@@ -118,6 +118,26 @@ msa_status_t msa_index_scores(const msa_config_t* cfg, const msa_batch_t* batch,
                               const void* idx_k_cache, float* block_scores, cudaStream_t stream);
 
 /*
+ * msa_index_scores over an FP8 indexer-key cache, for calls with at most 8
+ * queries per sequence (decode and verify; MSA_ERR_UNSUPPORTED otherwise).
+ * The pages list "FP8 KV-cache paths" among the upcoming work (daily.dev
+ * "MiniMax M3 ...", section "What's coming") and fix no format; this library
+ * reads e4m3 ("fn": finite range +-448, subnormals down to 2^-9) codes with
+ * one float scale for the whole cache:
+ *   idx_k_cache_e4m3  uint8 [num_pages][idx_heads][block_size][idx_dim], the
+ *                     e4m3 bit patterns; key value = code * k_scale
+ * (a writer stores e4m3(clamp(x / k_scale, -448, 448)), rounded to nearest
+ * even).  block_scores are those of msa_index_scores on the read-back keys:
+ *   block_scores[t][g][b] = sum_{h in heads(g)} max_{j in b, j <= p} idx_q[t][h] . (code[j][h] * k_scale)
+ * computed as k_scale times the fp32 dot products of the bf16 queries with the
+ * codes widened exactly.  k_scale must be positive and finite
+ * (MSA_ERR_INVALID_ARG otherwise).  Everything else as msa_index_scores.
+ */
+msa_status_t msa_index_scores_fp8(const msa_config_t* cfg, const msa_batch_t* batch, const void* idx_q,
+                                  const void* idx_k_cache_e4m3, float k_scale, float* block_scores,
+                                  cudaStream_t stream);
+
+/*
  * Top-k block selection per (query row, group).  cur = p / block_size is
  * always kept; the other topk-1 slots take the best blocks b < cur with a
  * finite score, ranked by (score descending, b ascending); a -inf score is
@@ -166,10 +186,11 @@ msa_status_t msa_attn_prefill(const msa_config_t* cfg, const msa_batch_t* batch,
 
 /*
  * Same result as msa_attn_prefill, organised for few queries per sequence:
- * one CTA per (row, group, split of the selected slots), online softmax
- * inside a split and a log-sum-exp merge of the splits.  `workspace` must
- * hold msa_decode_workspace_bytes(cfg, batch) bytes; its first
- * total_q * num_kv_heads int32 counters are cleared by the call itself.
+ * the selected slots of each (row, group) are split into runs of at most 8
+ * blocks, each run's blocks go through the tensor cores in swap-AB form and
+ * are combined by log-sum-exp, then a second kernel merges the runs the same
+ * way.  `workspace` must hold msa_decode_workspace_bytes(cfg, batch) bytes;
+ * nothing in it needs to be initialised.
  */
 msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, const void* q,
                              const void* k_cache, const void* v_cache, const int32_t* block_idx, void* out,
@@ -193,9 +214,9 @@ msa_status_t msa_attn_decode(const msa_config_t* cfg, const msa_batch_t* batch, 
  *   - `stream` must belong to the current device (MSA_ERR_INVALID_ARG
  *     otherwise), whose copy of the array the call uses.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents; the call clears the counters it needs.  Calls that can overlap
- *     on the GPU (different streams, or concurrent host threads) race on the
- *     array: serialize them.
+ *     contents; nothing in it needs to start at zero (every call writes what
+ *     it reads).  Calls that can overlap on the GPU (different streams, or
+ *     concurrent host threads) race on the array: serialize them.
  */
 msa_status_t msa_attn_decode_noalloc(const msa_config_t* cfg, const msa_batch_t* batch, const void* q,
                                      const void* k_cache, const void* v_cache, const int32_t* block_idx, void* out,

@@ -55,6 +55,18 @@ def quantize(x, scale: float) -> np.ndarray:
     return round_e4m3(_f64(x) / float(scale))
 
 
+def decode_bits(bits) -> np.ndarray:
+    """Values of e4m3 ("fn") bit patterns (uint8): sign bit 7, exponent bits 6..3 (bias 7), mantissa
+    bits 2..0; exponent 0 is subnormal (m * 2^-9); the two patterns 0x7F / 0xFF are NaN."""
+    b = np.asarray(bits, dtype=np.int64) & 0xFF
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64)))
+    mag = np.where((b & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
 def dequantize(codes, scale: float) -> np.ndarray:
     return _f64(codes) * float(scale)
 

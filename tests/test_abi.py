@@ -18,7 +18,7 @@ HEADER = os.path.join(ROOT, "include", "msa.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(msa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(msa_[a-z0-9_]+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -38,7 +38,7 @@ def test_header_declares_the_entry_points():
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", msa.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
-    exported = set(re.findall(r"\bT (msa_[a-z_]+)$", out, flags=re.M))
+    exported = set(re.findall(r"\bT (msa_[a-z0-9_]+)$", out, flags=re.M))
     missing = [n for n in declared_functions() if n not in exported]
     assert not missing, missing
     assert set(msa.EXPORTS) == set(declared_functions())

@@ -88,3 +88,16 @@ def test_pins_catch_plausible_slips():
     assert not np.array_equal(rounded(np.clip(x, -448, 448), "away"), want)
     assert not np.array_equal(rounded(np.clip(x, -448, 448), "trunc"), want)
     assert F.round_e4m3(np.array([1e6]))[0] == 448.0 != rounded(np.array([1e6]), "away")[0]
+
+
+def test_decode_bits_matches_torch_for_every_pattern():
+    bits = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(bits).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = F.decode_bits(bits)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    fin = ~np.isnan(want)
+    assert np.array_equal(got[fin], want[fin])
+    assert np.array_equal(np.signbit(got[fin]), np.signbit(want[fin]))   # -0 stays -0
+    # a planted slip (bias 8 instead of 7) fails
+    slip = np.where(((bits >> 3) & 0xF) == 0, got, got / 2)
+    assert not np.array_equal(slip[fin], want[fin])
