@@ -15,12 +15,10 @@
 // One CTA per row: its r/2 rotation angles are formed once, in double
 // precision (positions reach 2^20, where a float product p * theta^(-2i/r)
 // would be off by hundredths of a radian), and shared by all the row's heads.
-// A warp takes every 8th head of the row: lane l holds channels 4l .. 4l+3
-// (8-byte accesses), the sum of squares is a warp reduction, and the partner
-// of channel c < r/2 (channel c + r/2) sits r/8 lanes further on.  All of a
-// warp's head loads (and the row's page id) are issued before the angles are
-// ready, so the row costs one memory latency, not one per head.
-// Memory-bound: each head row is read once and written once.
+// A warp takes one head at a time: lane l holds channels 4l .. 4l+3 (one 8-byte
+// load), the sum of squares is a warp reduction, and the partner of channel
+// c < r/2 (channel c + r/2) sits r/8 lanes further on.  Memory-bound: each
+// head row is read once and written once.
 #pragma once
 #include "common.cuh"
 
@@ -56,26 +54,10 @@ __device__ __forceinline__ void store_bf16x4(__nv_bfloat16* p, const float (&x)[
   *reinterpret_cast<uint2*>(p) = w;
 }
 
-constexpr int QKR_MAXH = 9;     // heads per warp: ceil((64 + 4) / 8) for the 64 / 4 configuration; more loop
-
 __global__ void __launch_bounds__(QKR_THREADS) qk_rope_insert_kernel(const QkRopeArgs a) {
   __shared__ float s_cos[QKR_D / 2], s_sin[QKR_D / 2];
   const int t = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = QKR_THREADS / 32;
-  const int heads = a.Hq + a.Hkv;
-  const int c0 = 4 * lane;                       // this lane's channels c0 .. c0+3
-  auto src_of = [&](int j) -> const __nv_bfloat16* {
-    return j < a.Hq ? a.q + (static_cast<long>(t) * a.Hq + j) * QKR_D
-                    : a.k_new + (static_cast<long>(t) * a.Hkv + (j - a.Hq)) * QKR_D;
-  };
-  // every head of this warp in flight at once (heads warp, warp + 8, ...)
-  float xs[QKR_MAXH][4];
-#pragma unroll
-  for (int k = 0; k < QKR_MAXH; ++k) {
-    const int j = warp + k * NW;
-    if (j < heads) load_bf16x4(src_of(j) + c0, xs[k]);
-  }
   const int s = find_seq(a.q_start, a.num_seqs, t);
   const int qs = __ldg(a.q_start + s), nq = __ldg(a.q_start + s + 1) - qs;
   const int p = __ldg(a.ctx_len + s) - nq + (t - qs);
@@ -88,6 +70,8 @@ __global__ void __launch_bounds__(QKR_THREADS) qk_rope_insert_kernel(const QkRop
     s_cos[tid] = static_cast<float>(cs);
     s_sin[tid] = static_cast<float>(sn);
   }
+  __syncthreads();
+
   // the row's cache slot (checked once; a bad page skips the cache writes, never the queries)
   const int blk = p >= 0 ? p / a.block_size : -1;
   int page = -1;
@@ -95,26 +79,18 @@ __global__ void __launch_bounds__(QKR_THREADS) qk_rope_insert_kernel(const QkRop
   const bool page_ok = page >= 0 && page < a.num_pages;
   if (!page_ok && tid == 0) flag_error(MSA_DEV_BOUNDS);
   const int slot = p >= 0 ? p % a.block_size : 0;
-  __syncthreads();
 
+  const int c0 = 4 * lane;                       // this lane's channels c0 .. c0+3
   const int pd = half >> 2;                      // partner distance in lanes (r/8)
   const int partner = lane < pd ? lane + pd : (lane < 2 * pd ? lane - pd : lane);
-  float wq[4], wk[4];
-  load_bf16x4(a.q_w + c0, wq);
-  load_bf16x4(a.k_w + c0, wk);
-  for (int k = 0; k * NW + warp < heads; ++k) {  // uniform over the warp
-    const int j = warp + k * NW;
+  for (int j = warp; j < a.Hq + a.Hkv; j += QKR_THREADS / 32) {   // uniform over the warp
     const bool is_q = j < a.Hq;
     const int g = j - a.Hq;
-    float x[4];
-    if (k < QKR_MAXH) {
-#pragma unroll
-      for (int kk = 0; kk < QKR_MAXH; ++kk)
-        if (kk == k) { x[0] = xs[kk][0]; x[1] = xs[kk][1]; x[2] = xs[kk][2]; x[3] = xs[kk][3]; }
-    } else {
-      load_bf16x4(src_of(j) + c0, x);            // configurations with more heads than the prefetch holds
-    }
-    const float (&w)[4] = is_q ? wq : wk;
+    const __nv_bfloat16* src = is_q ? a.q + (static_cast<long>(t) * a.Hq + j) * QKR_D
+                                    : a.k_new + (static_cast<long>(t) * a.Hkv + g) * QKR_D;
+    float x[4], w[4];
+    load_bf16x4(src + c0, x);
+    load_bf16x4((is_q ? a.q_w : a.k_w) + c0, w);
     float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
