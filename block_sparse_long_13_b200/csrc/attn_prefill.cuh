@@ -627,16 +627,28 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeArgs a) {
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float wsum = 0.f;
   if (mx > -INFINITY) {
-    for (int s = 0; s < a.topk; ++s) {
-      if (__ldg(sel + s) < 0) continue;
-      const float w = __expf(__ldg(pl + s) - mx);
-      wsum += w;
-      const uint4 o = __ldg(reinterpret_cast<const uint4*>(
-          a.part_o + ((static_cast<long>(t) * a.topk + s) * a.Hq + head) * 128 + d8 * 8));
-      acc[0] = fmaf(w, bf16lo(o.x), acc[0]); acc[1] = fmaf(w, bf16hi(o.x), acc[1]);
-      acc[2] = fmaf(w, bf16lo(o.y), acc[2]); acc[3] = fmaf(w, bf16hi(o.y), acc[3]);
-      acc[4] = fmaf(w, bf16lo(o.z), acc[4]); acc[5] = fmaf(w, bf16hi(o.z), acc[5]);
-      acc[6] = fmaf(w, bf16lo(o.w), acc[6]); acc[7] = fmaf(w, bf16hi(o.w), acc[7]);
+    // 8 slots per round, every partial load of the round issued before the first is used
+    const __nv_bfloat16* po = a.part_o + (static_cast<long>(t) * a.topk * a.Hq + head) * 128 + d8 * 8;
+    for (int s0 = 0; s0 < a.topk; s0 += 8) {
+      uint4 o[8];
+      bool use[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int s = s0 + k;
+        use[k] = s < a.topk && __ldg(sel + s) >= 0;
+        o[k] = use[k] ? __ldcs(reinterpret_cast<const uint4*>(po + static_cast<long>(s) * a.Hq * 128))
+                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (!use[k]) continue;
+        const float w = __expf(__ldg(pl + s0 + k) - mx);
+        wsum += w;
+        acc[0] = fmaf(w, bf16lo(o[k].x), acc[0]); acc[1] = fmaf(w, bf16hi(o[k].x), acc[1]);
+        acc[2] = fmaf(w, bf16lo(o[k].y), acc[2]); acc[3] = fmaf(w, bf16hi(o[k].y), acc[3]);
+        acc[4] = fmaf(w, bf16lo(o[k].z), acc[4]); acc[5] = fmaf(w, bf16hi(o[k].z), acc[5]);
+        acc[6] = fmaf(w, bf16lo(o[k].w), acc[6]); acc[7] = fmaf(w, bf16hi(o[k].w), acc[7]);
+      }
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
