@@ -126,9 +126,15 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
     if (lane == 0) tma_prefetch_desc(&tmap_k);
     int page_l = 0;
     uint32_t used = 0, parity_bits = 0;   // per ring slot: issued at least once / parity of the last issue
+    // stage k = (unit j, group g) and its ring slot, kept as counters (no 64-bit division per stage)
+    long j = 0;
+    int g = 0, slot = 0;
+    uint32_t par = 0;
     for (long k = 0; k < nstage; ++k) {
-      const long j = k / a.Hkv;           // unit index within this CTA
-      const int g = static_cast<int>(k % a.Hkv);
+      if (k > 0) {
+        if (++g == a.Hkv) { g = 0; ++j; }
+        if (++slot == a.stages) { slot = 0; par ^= 1u; }
+      }
       if (g == 0 && (j & 31) == 0) {      // page ids of the next 32 units, one per lane
         const long uu = u0 + j + lane;
         page_l = 0;
@@ -140,8 +146,6 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
         }
       }
       const int page = __shfl_sync(0xFFFFFFFFu, page_l, static_cast<int>(j & 31));
-      const int slot = static_cast<int>(k % a.stages);
-      const uint32_t par = static_cast<uint32_t>((k / a.stages) & 1);
       bool ok = true;
       if (lane == 0) {
         ok = mbar_wait(&empty_bar[slot], par ^ 1u, &s_abort);
@@ -172,7 +176,6 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
     int cur_seq = -1, nq = 0, qrow0 = 0, ctx = 0;
     int s, b;
     locate(u0, s, b);
-    long cur_unit = 0;                    // unit (s, b) stands for, within this CTA
     // the per-group sum of the group's previous stage is made after the barrier that opens the next one
     int pv_nq = 0, pv_row0 = 0, pv_g = 0, pv_b = 0;
     auto combine = [&](int pbuf) {
@@ -188,12 +191,24 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
     };
     bool ok = true;
     int m = 0;                            // stages taken by this group so far
+    // stage k = (unit, group g) and its ring slot, kept as counters: a 64-bit division per stage would
+    // cost these threads as much as the stage's dot products
+    int g = 0, slot = 0;
+    uint32_t par = 0;
+    auto next_unit = [&]() {              // next block, or next sequence with blocks
+      ++b;
+      while (b >= s_nbprefix[s + 1] - s_nbprefix[s]) { ++s; b = 0; }
+    };
+    for (int d = 0; d < grp && grp < nstage; ++d) {   // this group starts at stage grp
+      if (++g == a.Hkv) { g = 0; next_unit(); }
+      if (++slot == a.stages) { slot = 0; par ^= 1u; }
+    }
     for (long k = grp; k < nstage; k += NG, ++m) {
-      const int g = static_cast<int>(k % a.Hkv);
-      for (const long unit = k / a.Hkv; cur_unit < unit; ++cur_unit) {   // next block, or next sequence with blocks
-        ++b;
-        while (b >= s_nbprefix[s + 1] - s_nbprefix[s]) { ++s; b = 0; }
-      }
+      if (m > 0)
+        for (int d = 0; d < NG; ++d) {
+          if (++g == a.Hkv) { g = 0; next_unit(); }
+          if (++slot == a.stages) { slot = 0; par ^= 1u; }
+        }
       if (s != cur_seq) {
         // this sequence's queries (all indexer heads) as fp32
         named_bar_sync(bar_seq, IDXD_CONSUMERS);
@@ -207,8 +222,6 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeA
         for (int i = cl; i < n; i += IDXD_CONSUMERS) s_q[i] = __bfloat162float(src[i]);
         named_bar_sync(bar_seq, IDXD_CONSUMERS);
       }
-      const int slot = static_cast<int>(k % a.stages);
-      const uint32_t par = static_cast<uint32_t>((k / a.stages) & 1);
       if (!mbar_wait_group(&full_bar[slot], par, &s_abort, bar_stage, IDXD_CONSUMERS)) { ok = false; break; }
       if (m > 0) combine((m - 1) & 1);
       const uint8_t* tile = ring + static_cast<long>(slot) * a.stage_bytes;

@@ -116,9 +116,15 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
     int cur_seq = -1, nseq = 0;
     uint32_t used = 0, parity_bits = 0;   // per ring slot: issued at least once / parity of the last issue
     bool ok = true;
+    // stage k = (unit j, group g) and its ring slot, kept as counters (no 64-bit division per stage)
+    long j = 0;
+    int g = 0, slot = 0;
+    uint32_t par = 0;
     for (long k = 0; k < nstage && ok; ++k) {
-      const long j = k / a.Hkv;           // unit index within this CTA
-      const int g = static_cast<int>(k % a.Hkv);
+      if (k > 0) {
+        if (++g == a.Hkv) { g = 0; ++j; }
+        if (++slot == a.stages) { slot = 0; par ^= 1u; }
+      }
       if (g == 0 && (j & 31) == 0) {      // page ids (and sequences) of the next 32 units, one per lane
         const long uu = u0 + j + lane;
         page_l = 0;
@@ -146,8 +152,6 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
           cur_seq = seq;
           ++nseq;
         }
-        const int slot = static_cast<int>(k % a.stages);
-        const uint32_t par = static_cast<uint32_t>((k / a.stages) & 1);
         if (ok) ok = mbar_wait(&empty_bar[slot], par ^ 1u, &s_abort);
         if (ok) {
           mbar_arrive_expect_tx(&full_bar[slot], a.stage_bytes);
@@ -170,22 +174,26 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
     const uint64_t qdesc0 = sdesc_sw128(smem_u32(q_s), 16, 1024);
     int s, b;
     locate(u0, s, b);
-    long cur_unit = 0;
     int cur_seq = -1, nseq = 0;
     bool ok = true;
+    int g = 0, slot = 0, as = 0;
+    uint32_t par = 0, apar = 0;
     for (long k = 0; k < nstage && ok && !s_abort; ++k) {
-      const int g = static_cast<int>(k % a.Hkv);
-      for (const long unit = k / a.Hkv; cur_unit < unit; ++cur_unit) advance(s, b);
+      if (k > 0) {
+        if (++g == a.Hkv) { g = 0; advance(s, b); }
+        if (++slot == a.stages) { slot = 0; par ^= 1u; }
+        if (++as == nslot) { as = 0; apar ^= 1u; }
+      }
       if (s != cur_seq) {
         if (cur_seq >= 0) umma_commit(&q_empty[(nseq - 1) & 1]);   // the previous sequence's queries are free
         if (!mbar_wait(&q_full[nseq & 1], (nseq >> 1) & 1, &s_abort)) break;
         cur_seq = s;
         ++nseq;
       }
-      const int slot = static_cast<int>(k % a.stages);
-      const int as = static_cast<int>(k % nslot);
-      if (!mbar_wait(&full_bar[slot], static_cast<uint32_t>((k / a.stages) & 1), &s_abort) ||
-          !mbar_wait(&acc_empty[as], static_cast<uint32_t>((k / nslot) & 1) ^ 1u, &s_abort)) { ok = false; break; }
+      if (!mbar_wait(&full_bar[slot], par, &s_abort) || !mbar_wait(&acc_empty[as], apar ^ 1u, &s_abort)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint64_t kd = kdesc0 + static_cast<uint64_t>((static_cast<long>(slot) * a.stage_bytes) >> 4);
       const uint64_t qd = qdesc0 + static_cast<uint64_t>((((nseq - 1) & 1) * q_bytes) >> 4);
@@ -211,7 +219,6 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     int s, b;
     locate(u0, s, b);
-    long cur_unit = 0;
     int cur_seq = -1, nq = 0, qrow0 = 0, ctx = 0;
     int pv_nq = 0, pv_row0 = 0, pv_g = 0, pv_b = 0;
     auto combine = [&](int pbuf) {                       // the previous stage's block scores
@@ -225,9 +232,13 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
       }
     };
     bool ok = true;
+    int g = 0, as = 0;
+    uint32_t apar = 0;
     for (long k = 0; k < nstage; ++k) {
-      const int g = static_cast<int>(k % a.Hkv);
-      for (const long unit = k / a.Hkv; cur_unit < unit; ++cur_unit) advance(s, b);
+      if (k > 0) {
+        if (++g == a.Hkv) { g = 0; advance(s, b); }
+        if (++as == nslot) { as = 0; apar ^= 1u; }
+      }
       if (s != cur_seq) {
         cur_seq = s;
         qrow0 = __ldg(a.q_start + s);
@@ -235,9 +246,8 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
         ctx = __ldg(a.ctx_len + s);
         if (nq > NQ) { if (ptid == 0) flag_error(MSA_DEV_BOUNDS); nq = NQ; }
       }
-      const int as = static_cast<int>(k % nslot);
       // the group wait is also the barrier after which the previous stage's partial maxima are visible
-      if (!mbar_wait_group(&acc_full[as], static_cast<uint32_t>((k / nslot) & 1), &s_abort, 1, 128)) {
+      if (!mbar_wait_group(&acc_full[as], apar, &s_abort, 1, 128)) {
         ok = false;
         break;
       }

@@ -300,9 +300,11 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
         for (int i = 1; i < IDXP_FUSED_SLOTS; ++i)
           if (ck[i] < kmin) { kmin = ck[i]; kpos = i; }
       };
+      // head hl of the group and this warpgroup's block b of step sp, kept as counters: a runtime
+      // division per step sits on this loop's dependency chain
+      int hl = 0, b = w;
       for (int sp = 0; sp < nstep; ++sp, ++ait) {
-        const int hl = sp % a.hg;
-        const int b = 2 * (sp / a.hg) + w;     // this warpgroup's block
+        if (sp > 0 && ++hl == a.hg) { hl = 0; b += 2; }
         const int buf = ait & 1;
         if (!mbar_wait_warp(&acc_full[buf], (ait >> 1) & 1, &s_abort)) { ok = false; break; }
         tc_fence_after();
