@@ -652,7 +652,12 @@ msa_status_t msa_qknorm_rope_insert(const msa_config_t* cfg, const msa_batch_t* 
   a.rotary_dim = rotary_dim;
   a.log2_theta = std::log2(static_cast<double>(rope_theta));
   a.eps = eps;
-  msa::qk_rope_insert_kernel<<<static_cast<unsigned>(batch->total_q), msa::QKR_THREADS, 0, stream>>>(a);
+  const int smem = msa::qkr_smem_bytes(a.Hq, a.Hkv);
+  CUDA_TRY(set_smem(msa::qk_rope_insert_kernel, smem));
+  // eight CTAs per SM need their shared memory more than L1 (no data is reused)
+  CUDA_TRY(cudaFuncSetAttribute(msa::qk_rope_insert_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared));
+  msa::qk_rope_insert_kernel<<<static_cast<unsigned>(batch->total_q), msa::QKR_THREADS, smem, stream>>>(a);
   return launched();
 }
 
