@@ -20,14 +20,19 @@
 // Persistent CTAs (one per SM) own contiguous runs of (sequence, block) units
 // as in the CUDA-core form; warp 0 streams the key tiles (and, when the
 // sequence changes, its query tile), warp 1 issues the MMAs into a ring of TMEM
-// accumulators, warps 2-5 pool.  Every wait is bounded.
+// accumulators, and two pooling groups (warps 2-5 and 6-9) take alternate
+// stages: one group's per-stage chain (TMEM read, warp maxima, the previous
+// stage's sums) is longer than the stream's time per stage.  Every wait is
+// bounded.
 #pragma once
 #include "common.cuh"
 #include "index_decode.cuh"
 
 namespace msa {
 
-constexpr int IDXT_THREADS = 192;
+constexpr int IDXT_GROUPS = 2;      // pooling groups of 4 warps, alternate stages
+constexpr int IDXT_THREADS = 64 + IDXT_GROUPS * 128;
+constexpr int IDXT_MAXHG = 4;       // indexer heads per KV group (the configuration allows at most 4)
 constexpr int IDXT_MAXQ = 16;       // query rows per sequence (the MMA's N)
 constexpr int IDXT_QHEAD = 2048;    // one head's query tile: 16 rows x 64 dims bf16, 128-byte swizzle
 
@@ -43,7 +48,7 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
   const int q_bytes = a.Hi * IDXT_QHEAD;
   __shared__ uint64_t full_bar[16], empty_bar[16], acc_full[8], acc_empty[8], q_full[2], q_empty[2], drain_bar;
   __shared__ int s_nbprefix[IDXD_MAXSEQ + 1];
-  __shared__ uint32_t s_part[2][NQ][IDXD_MAXHG][4];
+  __shared__ uint32_t s_part[2 * IDXT_GROUPS][NQ][IDXT_MAXHG][4];   // per group, this and the previous stage
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
 
@@ -213,15 +218,17 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
     }
   } else if (nstage > 0 && warp >= 2) {
     // ------------------------------------------------------------ pooling warps: thread = key row
+    // group G takes the stages k with k % IDXT_GROUPS == G; its 4 warps cover the 4 TMEM lane quarters
+    const int G = (warp - 2) >> 2;
     const int q4 = warp & 3;
     const int token = q4 * 32 + lane;
-    const int ptid = (warp - 2) * 32 + lane;             // 0..127
+    const int ptid = ((warp - 2) & 3) * 32 + lane;       // 0..127 within the group
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     int s, b;
     locate(u0, s, b);
     int cur_seq = -1, nq = 0, qrow0 = 0, ctx = 0;
     int pv_nq = 0, pv_row0 = 0, pv_g = 0, pv_b = 0;
-    auto combine = [&](int pbuf) {                       // the previous stage's block scores
+    auto combine = [&](int pbuf) {                       // the group's previous stage: block scores
       if (ptid < pv_nq) {
         float tot = 0.f;
         for (int hl = 0; hl < a.hg; ++hl) {
@@ -232,13 +239,14 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
       }
     };
     bool ok = true;
-    int g = 0, as = 0;
+    int g = 0, as = 0, done = 0;
     uint32_t apar = 0;
     for (long k = 0; k < nstage; ++k) {
       if (k > 0) {
         if (++g == a.Hkv) { g = 0; advance(s, b); }
         if (++as == nslot) { as = 0; apar ^= 1u; }
       }
+      if ((k % IDXT_GROUPS) != G) continue;
       if (s != cur_seq) {
         cur_seq = s;
         qrow0 = __ldg(a.q_start + s);
@@ -246,36 +254,43 @@ index_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,   // keys (64
         ctx = __ldg(a.ctx_len + s);
         if (nq > NQ) { if (ptid == 0) flag_error(MSA_DEV_BOUNDS); nq = NQ; }
       }
-      // the group wait is also the barrier after which the previous stage's partial maxima are visible
-      if (!mbar_wait_group(&acc_full[as], apar, &s_abort, 1, 128)) {
+      // the group wait is also the barrier after which the group's previous partial maxima are visible
+      if (!mbar_wait_group(&acc_full[as], apar, &s_abort, 1 + G, 128)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (k > 0) combine((k - 1) & 1);
-      const int pbuf = static_cast<int>(k & 1);
-      const int j = b * a.block_size + token;            // absolute key position
-      for (int hl = 0; hl < a.hg; ++hl) {
-        float v[16];
-        tmem_ld16(lane_addr + static_cast<uint32_t>((as * a.hg + hl) * 16), v);
-        tmem_ld_wait();
+      // every head's scores of this stage in flight at once, one wait
+      float v[IDXT_MAXHG][16];
 #pragma unroll
-        for (int i = 0; i < NQ; ++i) {
-          if (i < nq) {
-            const int p = ctx - nq + i;
-            const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, order_key(j <= p ? v[i] : -INFINITY));
-            if (lane == 0) s_part[pbuf][i][hl][q4] = mx;
-          }
-        }
-      }
+      for (int hl = 0; hl < IDXT_MAXHG; ++hl)
+        if (hl < a.hg) tmem_ld16(lane_addr + static_cast<uint32_t>((as * a.hg + hl) * 16), v[hl]);
+      if (done > 0) combine(((done - 1) & 1) * IDXT_GROUPS + G);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[as]);
+      const int pbuf = (done & 1) * IDXT_GROUPS + G;      // alternates over the group's own stages
+      const int j = b * a.block_size + token;            // absolute key position
+#pragma unroll
+      for (int hl = 0; hl < IDXT_MAXHG; ++hl) {
+        if (hl < a.hg) {
+#pragma unroll
+          for (int i = 0; i < NQ; ++i) {
+            if (i < nq) {
+              const int p = ctx - nq + i;
+              const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, order_key(j <= p ? v[hl][i] : -INFINITY));
+              if (lane == 0) s_part[pbuf][i][hl][q4] = mx;
+            }
+          }
+        }
+      }
       pv_nq = nq; pv_row0 = qrow0; pv_g = g; pv_b = b;
+      ++done;
     }
-    if (ok) {
-      named_bar_sync(1, 128);                            // the last stage's partial maxima visible
-      combine(static_cast<int>((nstage - 1) & 1));
+    if (ok && done > 0) {
+      named_bar_sync(1 + G, 128);                        // the group's last partial maxima visible
+      combine(((done - 1) & 1) * IDXT_GROUPS + G);
     }
   }
   __syncwarp();
