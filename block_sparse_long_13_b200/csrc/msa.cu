@@ -174,16 +174,18 @@ PrefillWs prefill_plan(const msa_config_t* c, const msa_batch_t* b) {
 }
 
 // Splits per (row, group) of the decode attention: a split holds at most msa::ATTD_MAXB selected
-// slots, and there should be about 2 work items per SM (more items share out more evenly, fewer
-// pay less per-item latency and merge traffic).
+// slots, and there should be about 6 work items per SM (the persistent CTAs then finish within
+// about one item of each other; 2 per SM left a quarter of the last round idle on 64 x 128K).  The
+// count is rounded so that every split holds the same number of slots (no empty trailing split).
 int decode_splits(const msa_config_t* c, const msa_batch_t* b) {
   const long units = static_cast<long>(b->total_q) * c->num_kv_heads;
   const long min_split = (c->topk + msa::ATTD_MAXB - 1) / msa::ATTD_MAXB;
   if (units <= 0) return static_cast<int>(min_split);
-  long want = (2L * 148 + units - 1) / units;
+  long want = (6L * 148 + units - 1) / units;
   want = std::max(want, min_split);
   want = std::min<long>(want, c->topk);
-  return static_cast<int>(want);
+  const long per = (c->topk + want - 1) / want;
+  return static_cast<int>((c->topk + per - 1) / per);
 }
 
 struct DecodeWs {
