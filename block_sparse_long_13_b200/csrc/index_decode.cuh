@@ -17,8 +17,9 @@
 // guarded by full/empty mbarriers.  The consumers are groups of 8 warps; a
 // group takes every NG-th stage (NG = 2 for at most 2 queries per sequence,
 // so one group's per-stage barrier and reduction latency hides behind the
-// other's work; else 1).  In a group each thread owns one key row, widens it
-// to fp32 and dots it with the sequence's (<= 8) queries held in shared
+// other's work, 3 for e4m3 keys and one query; else 1).  In a group each
+// thread owns one key row, widens it to fp32 and dots it with the
+// sequence's (<= 8) queries held in shared
 // memory; the block max is a warp redux.sync on order-preserving integer
 // keys, then a per-group sum over the heads.
 #pragma once
@@ -29,9 +30,15 @@
 namespace msa {
 
 constexpr int IDXD_CONSUMERS = 256;   // threads of one consumer group
-// consumer groups for a query bound NQ (the register budget of two groups fits NQ <= 2)
-__host__ __device__ constexpr int idxd_groups(int nq) { return nq <= 2 ? 2 : 1; }
-__host__ __device__ constexpr int idxd_threads(int nq) { return 32 + IDXD_CONSUMERS * idxd_groups(nq); }
+// consumer groups for a query bound NQ (the register budget of two groups fits NQ <= 2).  A group's
+// time per stage hardly depends on the stage's bytes, so e4m3 keys (half the bytes of a bf16 stage)
+// take three groups for one query per sequence.
+__host__ __device__ constexpr int idxd_groups(int nq, bool e4m3 = false) {
+  return nq <= 1 && e4m3 ? 3 : nq <= 2 ? 2 : 1;
+}
+__host__ __device__ constexpr int idxd_threads(int nq, bool e4m3 = false) {
+  return 32 + IDXD_CONSUMERS * idxd_groups(nq, e4m3);
+}
 constexpr int IDXD_MAXQ = 8;       // queries per sequence handled by this form
 constexpr int IDXD_MAXHG = 8;      // indexer heads per KV group
 constexpr int IDXD_MAXHI = 16;     // indexer heads
@@ -69,9 +76,9 @@ __device__ __forceinline__ void e4m3x16_to_f32(const uint4 w, float (&f)[16]) {
 // e4m3 codes (64-byte rows, 64-byte TMA swizzle) read back as code * k_scale; else bf16 (128-byte rows,
 // 128-byte swizzle).
 template <int NQ, bool E4M3 = false>
-__global__ void __launch_bounds__(idxd_threads(NQ), 1)
+__global__ void __launch_bounds__(idxd_threads(NQ, E4M3), 1)
 index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const IdxDecodeArgs a) {
-  constexpr int NG = idxd_groups(NQ);
+  constexpr int NG = idxd_groups(NQ, E4M3);
   extern __shared__ __align__(1024) uint8_t dsmem[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t full_bar[16], empty_bar[16];

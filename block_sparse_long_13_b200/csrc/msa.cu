@@ -358,13 +358,13 @@ msa_status_t launch_index_decode(const msa_config_t* cfg, const msa_batch_t* bat
     return go_tc(msa::index_decode_tc_kernel<8>);
   }
   const int nqb = mq <= 1 ? 1 : mq <= 2 ? 2 : mq <= 4 ? 4 : 8;   // compile-time query bound
-  const int q_bytes = msa::idxd_groups(nqb) * nqb * Hi * 64 * 4;   // each consumer group's queries
+  const int q_bytes = msa::idxd_groups(nqb, E4M3) * nqb * Hi * 64 * 4;   // each consumer group's queries
   a.stages = std::min(16, (msa::IDXD_SMEM_BUDGET - q_bytes) / a.stage_bytes);
   CHECK_SUP(a.stages >= 2, "indexer tiles too large for the shared-memory ring");
   const int smem = a.stages * a.stage_bytes + q_bytes + 1024;
   auto go = [&](auto kernel) -> msa_status_t {
     CUDA_TRY(set_smem(kernel, smem));
-    kernel<<<sms, msa::idxd_threads(nqb), smem, stream>>>(tk, a);
+    kernel<<<sms, msa::idxd_threads(nqb, E4M3), smem, stream>>>(tk, a);
     return launched();
   };
   if (mq <= 1) return go(msa::index_decode_kernel<1, E4M3>);

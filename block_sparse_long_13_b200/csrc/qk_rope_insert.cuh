@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(QKR_THREADS) qk_rope_insert_kernel(const QkRop
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(qkr_dsmem);   // [Hq + Hkv][128]: q heads, then k heads
   __nv_bfloat16* vs = xs + (a.Hq + a.Hkv) * QKR_D;                    // [Hkv][128]
   __shared__ float s_cos[QKR_D / 2], s_sin[QKR_D / 2];
-  __shared__ float s_w[2 * QKR_D];               // q_norm_w, then k_norm_w
+  __shared__ __align__(16) float s_w[2 * QKR_D];   // q_norm_w, then k_norm_w
   __shared__ uint64_t s_bar;
   __shared__ volatile int s_abort;
   const int t = blockIdx.x;
@@ -113,11 +113,11 @@ __global__ void __launch_bounds__(QKR_THREADS) qk_rope_insert_kernel(const QkRop
   const int ca = 4 * qa, cb = 4 * qb;
   if (tid < 2 * QKR_D) s_w[tid] = __bfloat162float(tid < QKR_D ? a.q_w[tid] : a.k_w[tid - QKR_D]);
   __syncthreads();                               // the barrier's init and the angles are visible
-  // every thread waits for the copies itself: a CTA never leaves while they are landing
-  if (!mbar_wait(&s_bar, 0, &s_abort)) {
-    if (tid == 0) mbar_wait_drain(&s_bar, 0);
-    return;
-  }
+  // one thread waits for the copies (the others sleep in the barrier instead of spinning on it); after
+  // a timed-out wait it lets them land before the CTA leaves
+  if (tid == 0 && !mbar_wait(&s_bar, 0, &s_abort)) mbar_wait_drain(&s_bar, 0);
+  __syncthreads();
+  if (s_abort) return;
   if (tid == 0 && page_ok) {                     // v rows go to the cache untouched
     for (int g = 0; g < a.Hkv; ++g) bulk_store(a.v_cache + kv_row + g * kv_head, vs + g * QKR_D, QKR_D * 2);
   }
@@ -144,11 +144,13 @@ __global__ void __launch_bounds__(QKR_THREADS) qk_rope_insert_kernel(const QkRop
     for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);   // within the half-warp
     const float inv = rsqrtf(ss * (1.f / QKR_D) + a.eps);
     const float* w = s_w + (is_q ? 0 : QKR_D);
+    const float4 w4a = *reinterpret_cast<const float4*>(w + ca), w4b = *reinterpret_cast<const float4*>(w + cb);
+    const float wa[4] = {w4a.x, w4a.y, w4a.z, w4a.w}, wb[4] = {w4b.x, w4b.y, w4b.z, w4b.w};
     float oa[4], ob[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float ya = xa[u] * inv * w[ca + u];
-      const float yb = xb[u] * inv * w[cb + u];
+      const float ya = xa[u] * inv * wa[u];
+      const float yb = xb[u] * inv * wb[u];
       // first of a pair: a cos - b sin; second: b cos + a sin (pass-through quads: cos 1, sin 0)
       oa[u] = rot ? ya * cs[u] - yb * sn[u] : ya;
       ob[u] = rot ? yb * cs[u] + ya * sn[u] : yb;
