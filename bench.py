@@ -107,17 +107,23 @@ class Part:
         self.pos = wl.positions()
 
     def run(self, ws, ev=None, stream=None, stop_after="attn"):
+        # NVTX ranges name each call of the part (part/index, part/topk, part/attn) for a profiler's timeline
         m = self.msa
+        nvtx = torch.cuda.nvtx
         if ev is not None:
             ev[0].record(stream)
+        nvtx.range_push(f"{self.name}/index")
         if self.fused:
             m.index_topk(self.cfg, self.batch, self.idx_q, self.caches["idx_k"], self.sel)
         else:
             m.index_scores(self.cfg, self.batch, self.idx_q, self.caches["idx_k"], self.scores)
+        nvtx.range_pop()
         if ev is not None:
             ev[1].record(stream)
         if stop_after != "index" and not self.fused:
+            nvtx.range_push(f"{self.name}/topk")
             m.topk_blocks(self.cfg, self.batch, self.scores, self.sel)
+            nvtx.range_pop()
         if ev is not None:
             ev[2].record(stream)
         if stop_after == "attn":
@@ -125,8 +131,10 @@ class Part:
             phases = ev is not None and self.kind == "prefill"
             if phases:
                 m.set_timing_events(ev[4:8])
+            nvtx.range_push(f"{self.name}/attn")
             fn(self.cfg, self.batch, self.q, self.caches["k"], self.caches["v"], self.sel, self.out, self.lse,
                ws[:self.ws_bytes])
+            nvtx.range_pop()
             if phases:
                 m.set_timing_events(None)
         if ev is not None:
