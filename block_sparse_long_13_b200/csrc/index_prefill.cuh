@@ -45,11 +45,13 @@ struct IdxPrefillArgs {
   const int32_t* page_table;
   int num_seqs, total_q, max_blocks, num_pages, Hi, Hkv, hg, block_size;
   int stages, nqbuf;         // key ring depth; query tile buffers
+  int nsplit;                // pieces per (query tile, group) along its key blocks (1 in the fused form)
 };
 
 struct IdxUnit {
-  int seq, row0, nrows, g, nblk;  // rows [row0, row0 + nrows); blocks 0 .. nblk-1
+  int seq, row0, nrows, g, nblk;  // rows [row0, row0 + nrows); the tile sees blocks 0 .. nblk-1
   int qs, nq, ctx;
+  int pr0, npr;                   // this piece: block pairs pr0 .. pr0+npr-1
 };
 
 // FUSED = false: write every block score.  FUSED = true: keep, per row, the best topk-1 earlier blocks
@@ -105,18 +107,23 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
   const uint32_t tmem = s_tmem;
 
   const int total_tiles = s_tprefix[a.num_seqs];
-  const int total_units = total_tiles * a.Hkv;
+  const long total_units = static_cast<long>(total_tiles) * a.Hkv * a.nsplit;
   const int G = gridDim.x;
 
-  // k-th unit of this CTA (snake order over the longest-first list); false when done
+  // k-th unit of this CTA (snake order over the longest-first list); false when done.  A unit is one of
+  // the nsplit pieces of a (query tile, group) along its key blocks: block scores need no reduction
+  // across blocks, and causal tiles differ in length, so whole tiles over the persistent CTAs left the
+  // last round 20-60 % unbalanced.
   auto get_unit = [&](int k, IdxUnit& u) -> bool {
     const int c = blockIdx.x;
     const long idx = static_cast<long>(k) * G + ((k & 1) ? (G - 1 - c) : c);
     if (idx >= total_units) return false;
+    const int piece = static_cast<int>(idx % a.nsplit);
+    const long tidx = idx / a.nsplit;
     // group-major: all CTAs work on one group's keys at a time (they stay in L2);
     // within a group the last (longest) query tiles come first
-    u.g = static_cast<int>(idx / total_tiles);
-    const int tau = total_tiles - 1 - static_cast<int>(idx % total_tiles);
+    u.g = static_cast<int>(tidx / total_tiles);
+    const int tau = total_tiles - 1 - static_cast<int>(tidx % total_tiles);
     int lo = 0, hi = a.num_seqs - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -132,6 +139,9 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
     const int p_last = u.ctx - u.nq + (u.row0 - u.qs) + u.nrows - 1;
     u.nblk = max(0, min(p_last / a.block_size + 1, a.max_blocks));
     if (p_last < 0) u.nblk = 0;
+    const int npair = (u.nblk + 1) >> 1;
+    u.pr0 = static_cast<int>(static_cast<long>(piece) * npair / a.nsplit);
+    u.npr = static_cast<int>(static_cast<long>(piece + 1) * npair / a.nsplit) - u.pr0;
     return true;
   };
 
@@ -150,7 +160,7 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
     int q_parity0 = -1, q_parity1 = -1;
     IdxUnit u;
     for (int k = 0; get_unit(k, u) && !s_abort; ++k) {
-      if (u.nblk == 0) continue;
+      if (u.npr == 0) continue;
       const int qb = uit % a.nqbuf;
       const uint32_t qpar = (uit / a.nqbuf) & 1;
       bool ok = true;
@@ -165,12 +175,11 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
       }
       if (__any_sync(0xFFFFFFFFu, !ok)) break;
       ++uit;
-      const int npair = (u.nblk + 1) >> 1;
       int page_l = 0;
-      for (int pr = 0; pr < npair && ok; ++pr) {
+      for (int pr = u.pr0; pr < u.pr0 + u.npr && ok; ++pr) {
         const int b0 = 2 * pr;
-        if ((b0 & 31) == 0) {                 // page ids of blocks b0 .. b0+31
-          const int bb = b0 + lane;
+        if ((b0 & 31) == 0 || pr == u.pr0) {  // page ids of the 32-block window holding b0 and b0+1
+          const int bb = (b0 & ~31) + lane;
           page_l = 0;
           if (bb < u.nblk) {
             page_l = __ldg(a.page_table + static_cast<long>(u.seq) * a.max_blocks + bb);
@@ -218,14 +227,14 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
     uint32_t uit = 0;
     IdxUnit u;
     for (int k = 0; get_unit(k, u) && !s_abort; ++k) {
-      if (u.nblk == 0) continue;
+      if (u.npr == 0) continue;
       const int qb = a.nqbuf == 1 ? 0 : static_cast<int>(uit & 1);
       const uint32_t qpar = a.nqbuf == 1 ? (uit & 1) : ((uit >> 1) & 1);
       if (!mbar_wait(&q_full[qb], qpar, &s_abort)) break;
       ++uit;
       // The tensor pipe queues about one MMA: the barriers of step sp + 1 are awaited while the first
       // two MMAs of step sp run, so the next step's MMAs are ready when the pipe frees up.
-      const int nstep = ((u.nblk + 1) >> 1) * a.hg;
+      const int nstep = u.npr * a.hg;
       bool ok = nstep > 0 && mbar_wait(&acc_empty[buf], (aph & 1) ^ 1, &s_abort) && mbar_wait(&k_full[st], kph, &s_abort);
       int hl = 0;
       for (int sp = 0; sp < nstep && ok; ++sp) {
@@ -271,12 +280,12 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
     uint32_t ait = 0;
     IdxUnit u;
     for (int k = 0; get_unit(k, u); ++k) {     // exits are warp-uniform
-      if (u.nblk == 0) continue;
+      if (u.npr == 0) continue;
       const bool valid = r < u.nrows;
       const int row = u.row0 + r;
       const int p = u.ctx - u.nq + (row - u.qs);
       float* srow = FUSED ? nullptr : a.scores + (static_cast<long>(row) * a.Hkv + u.g) * a.max_blocks;
-      const int nstep = ((u.nblk + 1) >> 1) * a.hg;
+      const int nstep = u.npr * a.hg;
       bool ok = true;
       float tot = 0.f;
       // fused form: candidate keys (order_key(score) << 32 | ~block); unused slots hold ~0 and are never
@@ -302,7 +311,7 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
       };
       // head hl of the group and this warpgroup's block b of step sp, kept as counters: a runtime
       // division per step sits on this loop's dependency chain
-      int hl = 0, b = w;
+      int hl = 0, b = 2 * u.pr0 + w;
       for (int sp = 0; sp < nstep; ++sp, ++ait) {
         if (sp > 0 && ++hl == a.hg) { hl = 0; b += 2; }
         const int buf = ait & 1;

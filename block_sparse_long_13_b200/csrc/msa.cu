@@ -258,6 +258,9 @@ msa_status_t launch_index_prefill(const msa_config_t* cfg, const msa_batch_t* ba
   a.Hkv = Hkv;
   a.hg = hg;
   a.block_size = cfg->block_size;
+  // pieces per (query tile, group) along its key blocks, for balance over the persistent CTAs; the fused
+  // form keeps each row's candidates over all of its blocks, so it takes whole tiles
+  a.nsplit = FUSED ? 1 : 4;
   const int q_tile = hg * 128 * 64 * 2;
   const int xbuf = FUSED ? 128 * msa::IDXP_FUSED_SLOTS * 8 : 0;   // candidate exchange between warpgroups
   a.nqbuf = (2 * q_tile + 2 * msa::IDXP_STAGE_BYTES <= 200 * 1024 - xbuf) ? 2 : 1;
