@@ -113,7 +113,7 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,   // idx_q  (64
   // k-th unit of this CTA (snake order over the longest-first list); false when done.  A unit is one of
   // the nsplit pieces of a (query tile, group) along its key blocks: block scores need no reduction
   // across blocks, and causal tiles differ in length, so whole tiles over the persistent CTAs left the
-  // last round 20-60 % unbalanced.
+  // last wave of units 20-60 % unbalanced.
   auto get_unit = [&](int k, IdxUnit& u) -> bool {
     const int c = blockIdx.x;
     const long idx = static_cast<long>(k) * G + ((k & 1) ? (G - 1 - c) : c);

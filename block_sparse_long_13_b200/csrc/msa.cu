@@ -175,7 +175,7 @@ PrefillWs prefill_plan(const msa_config_t* c, const msa_batch_t* b) {
 
 // Splits per (row, group) of the decode attention: a split holds at most msa::ATTD_MAXB selected
 // slots, and there should be about 6 work items per SM (the persistent CTAs then finish within
-// about one item of each other; 2 per SM left a quarter of the last round idle on 64 x 128K).  The
+// about one item of each other; 2 per SM left a quarter of the last wave idle on 64 x 128K).  The
 // count is rounded so that every split holds the same number of slots (no empty trailing split).
 int decode_splits(const msa_config_t* c, const msa_batch_t* b) {
   const long units = static_cast<long>(b->total_q) * c->num_kv_heads;
