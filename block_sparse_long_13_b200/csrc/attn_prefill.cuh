@@ -614,16 +614,25 @@ struct MergeArgs {
   int total_q, Hq, Hkv, topk;
 };
 
-// one CTA per (row, group): 16 heads x 16 threads x 8 output dims
+// one CTA per (row, group): 16 heads x 16 threads x 8 output dims.  The 16 threads of a head first read
+// the slots' selections and lse values in parallel (thread j: slots j, j + 16, ...), so the CTA pays one
+// round trip for them instead of one per slot, and leave each slot's weight in shared memory.
+constexpr int MRG_MAXK = 64;   // topk bound of the configuration
 __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeArgs a) {
+  __shared__ float s_w[ATTP_G][MRG_MAXK];   // per head and slot: exp(lse - max), or -1 (slot not selected)
   const int t = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
   const int h = threadIdx.x >> 4, d8 = threadIdx.x & 15;
   const int head = g * ATTP_G + h;
   const int32_t* sel = a.block_idx + (static_cast<long>(t) * a.Hkv + g) * a.topk;
   const float* pl = a.part_lse + (static_cast<long>(t) * a.Hq + head) * a.topk;
   float mx = -INFINITY;
-  for (int s = 0; s < a.topk; ++s)
+  for (int s = d8; s < a.topk; s += 16)
     if (__ldg(sel + s) >= 0) mx = fmaxf(mx, __ldg(pl + s));
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));   // the head's 16 lanes
+  for (int s = d8; s < a.topk; s += 16)
+    s_w[h][s] = __ldg(sel + s) >= 0 ? (mx > -INFINITY ? __expf(__ldg(pl + s) - mx) : 0.f) : -1.f;
+  __syncwarp();                             // a head's 16 threads share one warp
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float wsum = 0.f;
   if (mx > -INFINITY) {
@@ -631,23 +640,22 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeArgs a) {
     const __nv_bfloat16* po = a.part_o + (static_cast<long>(t) * a.topk * a.Hq + head) * 128 + d8 * 8;
     for (int s0 = 0; s0 < a.topk; s0 += 8) {
       uint4 o[8];
-      bool use[8];
+      float w[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int s = s0 + k;
-        use[k] = s < a.topk && __ldg(sel + s) >= 0;
-        o[k] = use[k] ? __ldcs(reinterpret_cast<const uint4*>(po + static_cast<long>(s) * a.Hq * 128))
-                      : make_uint4(0u, 0u, 0u, 0u);
+        w[k] = s < a.topk ? s_w[h][s] : -1.f;
+        o[k] = w[k] >= 0.f ? __ldcs(reinterpret_cast<const uint4*>(po + static_cast<long>(s) * a.Hq * 128))
+                           : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        if (!use[k]) continue;
-        const float w = __expf(__ldg(pl + s0 + k) - mx);
-        wsum += w;
-        acc[0] = fmaf(w, bf16lo(o[k].x), acc[0]); acc[1] = fmaf(w, bf16hi(o[k].x), acc[1]);
-        acc[2] = fmaf(w, bf16lo(o[k].y), acc[2]); acc[3] = fmaf(w, bf16hi(o[k].y), acc[3]);
-        acc[4] = fmaf(w, bf16lo(o[k].z), acc[4]); acc[5] = fmaf(w, bf16hi(o[k].z), acc[5]);
-        acc[6] = fmaf(w, bf16lo(o[k].w), acc[6]); acc[7] = fmaf(w, bf16hi(o[k].w), acc[7]);
+        if (w[k] < 0.f) continue;
+        wsum += w[k];
+        acc[0] = fmaf(w[k], bf16lo(o[k].x), acc[0]); acc[1] = fmaf(w[k], bf16hi(o[k].x), acc[1]);
+        acc[2] = fmaf(w[k], bf16lo(o[k].y), acc[2]); acc[3] = fmaf(w[k], bf16hi(o[k].y), acc[3]);
+        acc[4] = fmaf(w[k], bf16lo(o[k].z), acc[4]); acc[5] = fmaf(w[k], bf16hi(o[k].z), acc[5]);
+        acc[6] = fmaf(w[k], bf16lo(o[k].w), acc[6]); acc[7] = fmaf(w[k], bf16hi(o[k].w), acc[7]);
       }
     }
   }
