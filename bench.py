@@ -714,6 +714,8 @@ def main():
         k["flops"] += flops
         k["bytes"] += bytes_
 
+    decode_attn_parts = {}
+    name_of = {id(c): n for n, c in calls.items()}
     for c in calls.values():
         if c["kind"] == "prefill":
             if c["fused"]:
@@ -730,6 +732,9 @@ def main():
             addk("index_decode_kernel", c["index_ms"], 1, bytes_=c["index"]["bytes"])
             addk("topk kernel (decode)", c["topk_ms"], 1, bytes_=c["topk"]["bytes"])
             addk("attn_decode_kernel", c["attn_ms"], 1, bytes_=c["attn"]["bytes"])
+            if c["attn_ms"] > 0:   # each decode workload's attention on its own (the 8 x 1M one is a few us)
+                gbs = c["attn"]["bytes"] / c["attn_ms"] / 1e6
+                decode_attn_parts[name_of[id(c)]] = {"ms": c["attn_ms"], "gbs": gbs}
     # every kernel is timed inside a step of tens of ms, far shorter than the seconds-long loop the
     # sustained figure comes from: the burst tensor peak is the denominator
     tensor_peak, tensor_src = pk["bf16_tflops"], pk["source"] + " burst bf16 (cuBLAS)"
@@ -747,6 +752,9 @@ def main():
                                "frac": ach / pk["hbm_gbs"]}
         else:
             fractions[name] = {"ms_per_step": k["ms"], "launches_per_step": k["launches"]}
+    if "attn_decode_kernel" in fractions and decode_attn_parts:
+        fractions["attn_decode_kernel"]["per_part"] = {
+            n: dict(v, frac=v["gbs"] / pk["hbm_gbs"]) for n, v in decode_attn_parts.items()}
     dom_name, dom = max(((n, k) for n, k in kern.items() if k["flops"] > 0 or k["bytes"] > 0),
                         key=lambda nk: nk[1]["ms"])
     launch_ms = dom["ms"] / dom["launches"]
