@@ -426,6 +426,31 @@ class _Blocks:
         return x[sl.start - b * self.bs:sl.stop - b * self.bs]
 
 
+class _HostBlocks:
+    """Blocks already fetched to host arrays, sliced like the sequence they come from."""
+
+    def __init__(self, blocks, bs):
+        self.blocks, self.bs = blocks, bs
+
+    def __getitem__(self, sl):
+        b = sl.start // self.bs
+        x = self.blocks[b]
+        return x[sl.start - b * self.bs:sl.stop - b * self.bs]
+
+
+class _GenTokens:
+    """Token-order view of one sequence straight from the seeded generator: a slice generates only
+    its own tokens (the attention reads just the selected blocks; the whole 1M-token K and V of a
+    sequence would be 4 GB of float32 per sampled sequence)."""
+
+    def __init__(self, wl, tid, s, dev):
+        self.wl, self.tid, self.s, self.dev, self.ctx = wl, tid, s, dev, wl.ctx_len[s]
+
+    def __getitem__(self, sl):
+        idx = torch.arange(sl.start, min(sl.stop, self.ctx))
+        return gen.token_tensor(self.wl, self.tid, self.s, idx, device=self.dev).float().cpu().numpy()
+
+
 def _seq_tokens(wl, tid, s, cache=None, dev="cpu"):
     """float32 [ctx][H][D] of one sequence in token order: from the device cache when given
     (pages gathered), else from the seeded generator."""
@@ -444,6 +469,8 @@ class OracleLeg:
     of the step's workloads; the step's oracle time is extrapolated from each workload's time per
     query row.  Inputs come from the device caches of the timed step when there are any, else
     from the seeded generator (on the GPU when there is one); preparing them is not timed."""
+
+    GEN_POOL = 4   # decode sequences sampled per workload when inputs come from the generator
 
     def __init__(self, parts=None):
         from oracle import cpp as C
@@ -499,7 +526,7 @@ class OracleLeg:
         cc = p.caches if p is not None else None
         key = (name, s)
         if key not in self._decode:
-            if len(self._decode) > 2:
+            if len(self._decode) >= (2 * self.GEN_POOL if not self.parts else 3):
                 self._decode.clear()
             self._decode[key] = _seq_tokens(wl, gen.TID_IDX_K, s, cc["idx_k"] if cc else None, self.dev)
         ik = self._decode[key]
@@ -507,18 +534,26 @@ class OracleLeg:
         if cc is not None:
             k, v = _Blocks(cc["k"], wl.page_table[s, :nb]), _Blocks(cc["v"], wl.page_table[s, :nb])
         else:
-            k = gen.token_tensor(wl, gen.TID_K, s, torch.arange(wl.ctx_len[s]), device=self.dev).float().cpu().numpy()
-            v = gen.token_tensor(wl, gen.TID_V, s, torch.arange(wl.ctx_len[s]), device=self.dev).float().cpu().numpy()
+            k, v = _GenTokens(wl, gen.TID_K, s, self.dev), _GenTokens(wl, gen.TID_V, s, self.dev)
         rows = list(range(wl.q_start[s], wl.q_start[s + 1]))
         pos = wl.positions()[rows].numpy()
         q = gen.query_rows(wl, gen.TID_Q, device=self.dev)[rows].float().cpu().numpy() if p is None else \
             p.q[rows].float().cpu().numpy()
         iq = gen.query_rows(wl, gen.TID_IDX_Q, device=self.dev)[rows].float().cpu().numpy() if p is None else \
             p.idx_q[rows].float().cpu().numpy()
+        # timed: the oracle's three steps; not timed: fetching the selected K / V blocks (device cache
+        # or generator) into host arrays between the selection and the attention
         t0 = time.perf_counter()
-        s64, sel, out, lse = self.C.msa_rows(q, iq, k, v, ik, pos, wl.num_kv_heads, wl.block_size, wl.topk,
-                                             wl.max_blocks)
-        dt = time.perf_counter() - t0
+        s64 = self.C.block_scores(iq, ik, pos, wl.num_kv_heads, wl.block_size, wl.max_blocks)
+        sel = self.C.select_blocks(s64.astype(np.float32), pos, wl.topk, wl.block_size)
+        t1 = time.perf_counter()
+        bs = wl.block_size
+        blocks = sorted(set(int(b) for b in sel[sel >= 0].reshape(-1)))
+        kh = _HostBlocks({b: k[b * bs:(b + 1) * bs] for b in blocks}, bs)
+        vh = _HostBlocks({b: v[b * bs:(b + 1) * bs] for b in blocks}, bs)
+        t2 = time.perf_counter()
+        out, lse = self.C.sparse_attention(q, kh, vh, pos, sel, bs)
+        dt = (t1 - t0) + (time.perf_counter() - t2)
         if p is not None:
             for i, r in enumerate(rows):
                 self._compare(p, r, s64[i:i + 1], sel[i:i + 1], out[i:i + 1], pos[i:i + 1])
@@ -556,9 +591,12 @@ class OracleLeg:
         used["prefill_128k"], n_rows["prefill_128k"] = t_pre, n_pre
         for name, share in (("decode_128k", 0.3), ("decode_1m", 0.2)):
             wl_n = configs.ALL[name]().num_seqs
+            # without the step's device caches (the reference arm) every sampled sequence's indexer keys
+            # are generated again: a fixed few sequences, kept between steps (all have the same length)
+            pool = wl_n if self.parts else min(self.GEN_POOL, wl_n)
             t, n, s = 0.0, 0, 0
-            while (t < share * seconds or n == 0) and s < wl_n:
-                dt, k = self.decode_seq(name, int(self.rng.integers(0, wl_n)))
+            while (t < share * seconds or n == 0) and s < pool:
+                dt, k = self.decode_seq(name, int(self.rng.integers(0, pool)))
                 t, n, s = t + dt, n + k, s + 1
             per_row[name] = t / n
             used[name], n_rows[name] = t, n
